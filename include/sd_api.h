@@ -1,0 +1,248 @@
+/*
+ * sd_api.h -- C ABI of the B200 (sm_100a) Stable-Diffusion U-Net denoiser library.
+ *
+ * One forward pass of a Stable-Diffusion-style U-Net denoiser timestep at batch 1
+ * in BF16: ResnetBlock2D and Transformer2DModel blocks composed into the
+ * Down / Mid / Up topology with skip concatenation, stride-2 downsampling and
+ * nearest-2x upsampling.
+ *
+ * Sources (page title, section):
+ *   [SD21]  "Stable Diffusion 2.1 Base 宏观架构": section 3 (full U-Net multi-scale
+ *           topology: levels, skips, Conv_in 4->320, Conv_out 320->4), section 4
+ *           (core operators: ResnetBlock2D and Transformer2DModel panels).
+ *   [SDXLI] "Stable Diffusion XL Inpainting 宏观架构": sections 1-4 (9-channel
+ *           input = noisy latent + masked latent + mask; context [1,77,2048]).
+ *   [TUT]   SD/SDXL tutorial page (bfzx365.com, video 67462879): GSC bullet
+ *           (GroupNorm + SiLU + Conv), FeedForward bullet (GEGLU), DownSample
+ *           bullet (Conv k3 s2 p1), UpSample bullet (nearest + Conv k3 s1 p1),
+ *           BasicTransformer Block bullet, Spatial Transformer bullets, the
+ *           ResNetBlock paragraph and the sinusoidal time-embedding paragraph.
+ *   [SD15]  SD1.5 anatomy page (hotelren.com), section 3.4: Softmax(QK^T/sqrt(d))V.
+ *
+ * Conventions shared by every entry point
+ *   - Batch is 1. Activations are NHWC BF16, i.e. a token matrix [H*W, C] in
+ *     row-major pixel order (y*W + x). Context is BF16 [ctx_len, ctx_dim].
+ *   - Every device pointer is caller-owned device memory. The library never
+ *     allocates, frees or synchronises inside a *_fwd / sd_unet_step call; all
+ *     work is enqueued on the given stream, in order.
+ *   - Device pointers must be 16-byte aligned (SD_ERR_MISALIGNED otherwise).
+ *     Outputs must not alias inputs unless an entry point says otherwise.
+ *   - Weights are a packed BF16 buffer in the library's layout: obtain the
+ *     canonical tensor table with sd_*_weight_layout(), fill a canonical buffer
+ *     (tensors in table order, row-major in the canonical shapes, no padding),
+ *     convert it with sd_*_pack_weights() on the host and copy the result to the
+ *     device.
+ *   - All argument, shape, alignment and workspace checks run on the host before
+ *     any launch; on error nothing is launched and a status is returned. No call
+ *     aborts, prints or throws. Device-side waits are bounded; one that gives up
+ *     sets a flag in the workspace header that sd_query_device_status() reports.
+ *   - Thread safety: calls are re-entrant when they use distinct workspaces. The
+ *     only shared state is a per-device attribute cache guarded by a mutex.
+ */
+#ifndef SD_API_H
+#define SD_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* sd_stream_t; /* a cudaStream_t; NULL = the legacy default stream */
+
+typedef enum {
+  SD_OK = 0,
+  SD_ERR_NULL_ARG = 1,             /* a required pointer is NULL */
+  SD_ERR_BAD_SHAPE = 2,            /* inconsistent sizes, channel or context mismatch */
+  SD_ERR_UNSUPPORTED = 3,          /* batch != 1, head_dim != 64, C % 64 != 0, groups ... */
+  SD_ERR_MISALIGNED = 4,           /* a device pointer is not 16-byte aligned */
+  SD_ERR_WORKSPACE_TOO_SMALL = 5,  /* ws_bytes below sd_*_workspace_size() */
+  SD_ERR_NOT_SM100 = 6,            /* current device is not compute capability 10.0 */
+  SD_ERR_LAUNCH = 7,               /* a kernel launch or CUDA runtime call failed */
+  SD_ERR_DEVICE_TIMEOUT = 8,       /* a bounded device-side wait gave up */
+  SD_ERR_CAPACITY = 9              /* caller-provided table too small */
+} sd_status;
+
+/* Tensor kinds in a weight table. */
+enum { SD_KIND_WEIGHT = 0, SD_KIND_BIAS = 1, SD_KIND_NORM_GAMMA = 2, SD_KIND_NORM_BETA = 3 };
+
+typedef struct {
+  char name[80];          /* e.g. "down.0.res.1.conv1.weight" */
+  int32_t ndim;
+  int64_t shape[4];       /* canonical shape: conv [O, C, k, k], linear [out, in], vectors [n] */
+  int32_t kind;           /* SD_KIND_* */
+  int32_t fan_in;         /* C*k*k for conv, in_features for linear, 0 for norms */
+  int64_t canon_offset;   /* element offset in the canonical buffer */
+  int64_t packed_offset;  /* byte offset in the packed buffer */
+} sd_tensor_desc;
+
+/* ---------------------------------------------------------------- configurations */
+
+/* Time embedding MLP [TUT, time-embedding paragraph]: phi(t) sinusoid of
+ * proj_dim (cos half first, frequencies 10000^(-i/(proj_dim/2))), then
+ * Linear proj_dim->temb_dim, SiLU, Linear temb_dim->temb_dim. */
+typedef struct {
+  int32_t proj_dim;  /* 320 */
+  int32_t temb_dim;  /* 1280 */
+} sd_time_cfg;
+
+/* Plain convolutions: conv_in (3x3, c_in 4 or 9 -> c_out), downsample (3x3
+ * stride 2 pad 1, c_in = c_out), upsample (nearest 2x then 3x3), and the output
+ * head (GroupNorm + SiLU + 3x3 conv_out). height/width are the INPUT size. */
+typedef struct {
+  int32_t batch;   /* must be 1 */
+  int32_t height;
+  int32_t width;
+  int32_t c_in;
+  int32_t c_out;
+  int32_t groups;  /* output head only (32) */
+  float eps;       /* output head only (1e-5) */
+} sd_conv_cfg;
+
+/* ResnetBlock2D [SD21 section 4; TUT ResNetBlock paragraph]. Input is
+ * concat_C(x, skip) when c_skip > 0 (x channels first). A 1x1 shortcut conv is
+ * used when c_x + c_skip != c_out, else the identity. */
+typedef struct {
+  int32_t batch;     /* must be 1 */
+  int32_t height;
+  int32_t width;
+  int32_t c_x;       /* channels of x */
+  int32_t c_skip;    /* channels of the concatenated skip tensor, 0 = none */
+  int32_t c_out;
+  int32_t temb_dim;  /* 1280 */
+  int32_t groups;    /* 32 */
+  float eps;         /* 1e-5 */
+} sd_resblock_cfg;
+
+/* Transformer2DModel [SD21 section 4; TUT Spatial Transformer and
+ * BasicTransformer Block bullets]: GN -> proj_in -> depth x (LN -> self-attn,
+ * LN -> cross-attn on the context, LN -> GEGLU FF; each residual) -> proj_out,
+ * plus the block input. */
+typedef struct {
+  int32_t batch;     /* must be 1 */
+  int32_t height;
+  int32_t width;
+  int32_t channels;  /* C, a multiple of 64 */
+  int32_t head_dim;  /* must be 64; heads = C / 64 */
+  int32_t depth;     /* number of BasicTransformer blocks (1, 2, 10) */
+  int32_t ctx_len;   /* 1 .. 256 (77) */
+  int32_t ctx_dim;   /* 1024 or 2048 (multiple of 64) */
+  int32_t groups;    /* 32 */
+  float gn_eps;      /* 1e-5 */
+  float ln_eps;      /* 1e-5 */
+} sd_transformer_cfg;
+
+/* Whole denoiser [SD21 section 3; SDXLI section 3]. */
+typedef struct {
+  int32_t in_channels;        /* 4, or 9 for inpainting */
+  int32_t out_channels;       /* 4 */
+  int32_t height;             /* latent height, divisible by 2^(n_levels-1) */
+  int32_t width;
+  int32_t n_levels;           /* 1..4 */
+  int32_t block_channels[4];  /* 320, 640, 1280, 1280 */
+  int32_t attn_depth[4];      /* 1, 1, 1, 0 (0 = no transformer at that level) */
+  int32_t layers_per_block;   /* 2 (the up path uses layers_per_block + 1) */
+  int32_t mid_depth;          /* 1 */
+  int32_t head_dim;           /* 64 */
+  int32_t ctx_len;            /* 77 */
+  int32_t ctx_dim;            /* 1024 */
+  int32_t time_proj_dim;      /* 320 */
+  int32_t temb_dim;           /* 1280 */
+  int32_t groups;             /* 32 */
+  float eps;                  /* 1e-5, for every GroupNorm and LayerNorm */
+} sd_unet_cfg;
+
+/* ---------------------------------------------------------------- weights (host only) */
+
+/* Enumerate the canonical tensor table. `out` may be NULL (sizes only); when
+ * not NULL it must hold `capacity` entries (SD_ERR_CAPACITY otherwise, with
+ * *n_tensors still set). canon_elems: BF16 elements of the canonical buffer;
+ * packed_bytes: size of the packed buffer. Pure host code, no GPU needed. */
+sd_status sd_time_weight_layout(const sd_time_cfg* cfg, sd_tensor_desc* out, int32_t capacity,
+                                int32_t* n_tensors, int64_t* canon_elems, int64_t* packed_bytes);
+sd_status sd_conv_weight_layout(const sd_conv_cfg* cfg, int32_t conv_kind, sd_tensor_desc* out,
+                                int32_t capacity, int32_t* n_tensors, int64_t* canon_elems,
+                                int64_t* packed_bytes);
+sd_status sd_resblock_weight_layout(const sd_resblock_cfg* cfg, sd_tensor_desc* out, int32_t capacity,
+                                    int32_t* n_tensors, int64_t* canon_elems, int64_t* packed_bytes);
+sd_status sd_transformer_weight_layout(const sd_transformer_cfg* cfg, sd_tensor_desc* out,
+                                       int32_t capacity, int32_t* n_tensors, int64_t* canon_elems,
+                                       int64_t* packed_bytes);
+sd_status sd_unet_weight_layout(const sd_unet_cfg* cfg, sd_tensor_desc* out, int32_t capacity,
+                                int32_t* n_tensors, int64_t* canon_elems, int64_t* packed_bytes);
+
+/* conv_kind for sd_conv_weight_layout / sd_conv_pack_weights / sd_conv_fwd. */
+enum { SD_CONV_IN = 0, SD_CONV_DOWNSAMPLE = 1, SD_CONV_UPSAMPLE = 2, SD_CONV_OUTPUT = 3 };
+
+/* Convert a canonical BF16 buffer (host, uint16 bit patterns) into the packed
+ * layout (host buffer of packed_bytes). Conv weights become [O][ky][kx][C]; the
+ * GEGLU FF1 rows are interleaved (value j, gate j); everything else is copied.
+ * Each tensor starts on a 256-byte boundary. */
+sd_status sd_time_pack_weights(const sd_time_cfg* cfg, const uint16_t* canonical, void* packed);
+sd_status sd_conv_pack_weights(const sd_conv_cfg* cfg, int32_t conv_kind, const uint16_t* canonical,
+                               void* packed);
+sd_status sd_resblock_pack_weights(const sd_resblock_cfg* cfg, const uint16_t* canonical, void* packed);
+sd_status sd_transformer_pack_weights(const sd_transformer_cfg* cfg, const uint16_t* canonical,
+                                      void* packed);
+sd_status sd_unet_pack_weights(const sd_unet_cfg* cfg, const uint16_t* canonical, void* packed);
+
+/* ---------------------------------------------------------------- workspace sizes */
+
+size_t sd_time_workspace_size(const sd_time_cfg* cfg);
+size_t sd_conv_workspace_size(const sd_conv_cfg* cfg, int32_t conv_kind);
+size_t sd_resblock_workspace_size(const sd_resblock_cfg* cfg);
+size_t sd_transformer_workspace_size(const sd_transformer_cfg* cfg);
+size_t sd_unet_workspace_size(const sd_unet_cfg* cfg);
+
+/* ---------------------------------------------------------------- forward calls (device) */
+
+/* temb_out: device FP32 [temb_dim], the MLP output before any SiLU. */
+sd_status sd_time_embed(const sd_time_cfg* cfg, const void* packed_w, float timestep, float* temb_out,
+                        void* workspace, size_t ws_bytes, sd_stream_t stream);
+
+/* SD_CONV_IN: x0 = latent [H, W, c_in] BF16, or for c_in = 9 the inpaint input
+ *   assembled from x0 = noisy [H, W, 4], x1 = masked latent [H, W, 4],
+ *   x2 = mask [H, W, 1] (channels in that order) without materialising it.
+ *   y = [H, W, c_out].
+ * SD_CONV_DOWNSAMPLE: x0 = [H, W, C] -> y = [H/2, W/2, C] (3x3, stride 2, pad 1).
+ * SD_CONV_UPSAMPLE: x0 = [H, W, C] -> y = [2H, 2W, C] (nearest 2x, then 3x3).
+ * SD_CONV_OUTPUT: x0 = [H, W, C] -> y = [H, W, c_out] = conv_out(SiLU(GN(x0))). */
+sd_status sd_conv_fwd(const sd_conv_cfg* cfg, int32_t conv_kind, const void* packed_w, const void* x0,
+                      const void* x1, const void* x2, void* y, void* workspace, size_t ws_bytes,
+                      sd_stream_t stream);
+
+/* x [H, W, c_x], skip [H, W, c_skip] or NULL, temb device FP32 [temb_dim]
+ * (pre-SiLU MLP output), y [H, W, c_out]. */
+sd_status sd_resblock_fwd(const sd_resblock_cfg* cfg, const void* packed_w, const void* x,
+                          const void* skip, const float* temb, void* y, void* workspace, size_t ws_bytes,
+                          sd_stream_t stream);
+
+/* x [H, W, C], context [ctx_len, ctx_dim], y [H, W, C]. */
+sd_status sd_transformer_fwd(const sd_transformer_cfg* cfg, const void* packed_w, const void* x,
+                             const void* context, void* y, void* workspace, size_t ws_bytes,
+                             sd_stream_t stream);
+
+/* One denoiser timestep. latent: [H, W, in_channels] BF16 (for in_channels = 9
+ * the caller passes the assembled 9-channel input), context [ctx_len, ctx_dim],
+ * eps_out [H, W, out_channels]. The skip stack and every intermediate live in
+ * the workspace. */
+sd_status sd_unet_step(const sd_unet_cfg* cfg, const void* packed_w, const void* latent, float timestep,
+                       const void* context, void* eps_out, void* workspace, size_t ws_bytes,
+                       sd_stream_t stream);
+
+/* Synchronises `stream`, then reads the device error word of `workspace`:
+ * SD_OK, or SD_ERR_DEVICE_TIMEOUT when a bounded wait gave up; the word is
+ * cleared afterwards. */
+sd_status sd_query_device_status(void* workspace, sd_stream_t stream);
+
+const char* sd_status_string(sd_status s);
+
+/* Library version string ("sd-b200 <major>.<minor>"). */
+const char* sd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SD_API_H */

@@ -1,0 +1,302 @@
+"""ctypes binding of the C ABI declared in include/sd_api.h.
+
+Argument marshalling only: every function here has the name of the C entry
+point it calls and passes plain pointers and sizes through. The CUDA library
+must be built (``python -m latent_diffusion_net_b200.build``); loading fails
+loudly when it is missing. There is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char, c_char_p, c_float, c_int32, c_int64, c_size_t, c_uint16, c_void_p
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsd_b200.so")
+
+SD_OK = 0
+STATUS_NAMES = {0: "SD_OK", 1: "SD_ERR_NULL_ARG", 2: "SD_ERR_BAD_SHAPE", 3: "SD_ERR_UNSUPPORTED",
+                4: "SD_ERR_MISALIGNED", 5: "SD_ERR_WORKSPACE_TOO_SMALL", 6: "SD_ERR_NOT_SM100",
+                7: "SD_ERR_LAUNCH", 8: "SD_ERR_DEVICE_TIMEOUT", 9: "SD_ERR_CAPACITY"}
+SD_KIND_WEIGHT, SD_KIND_BIAS, SD_KIND_NORM_GAMMA, SD_KIND_NORM_BETA = 0, 1, 2, 3
+KIND_NAMES = {0: "weight", 1: "bias", 2: "norm_gamma", 3: "norm_beta"}
+SD_CONV_IN, SD_CONV_DOWNSAMPLE, SD_CONV_UPSAMPLE, SD_CONV_OUTPUT = 0, 1, 2, 3
+
+
+class SdError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+class sd_tensor_desc(ctypes.Structure):
+    _fields_ = [("name", c_char * 80), ("ndim", c_int32), ("shape", c_int64 * 4), ("kind", c_int32),
+                ("fan_in", c_int32), ("canon_offset", c_int64), ("packed_offset", c_int64)]
+
+
+class sd_time_cfg(ctypes.Structure):
+    _fields_ = [("proj_dim", c_int32), ("temb_dim", c_int32)]
+
+
+class sd_conv_cfg(ctypes.Structure):
+    _fields_ = [("batch", c_int32), ("height", c_int32), ("width", c_int32), ("c_in", c_int32),
+                ("c_out", c_int32), ("groups", c_int32), ("eps", c_float)]
+
+
+class sd_resblock_cfg(ctypes.Structure):
+    _fields_ = [("batch", c_int32), ("height", c_int32), ("width", c_int32), ("c_x", c_int32),
+                ("c_skip", c_int32), ("c_out", c_int32), ("temb_dim", c_int32), ("groups", c_int32),
+                ("eps", c_float)]
+
+
+class sd_transformer_cfg(ctypes.Structure):
+    _fields_ = [("batch", c_int32), ("height", c_int32), ("width", c_int32), ("channels", c_int32),
+                ("head_dim", c_int32), ("depth", c_int32), ("ctx_len", c_int32), ("ctx_dim", c_int32),
+                ("groups", c_int32), ("gn_eps", c_float), ("ln_eps", c_float)]
+
+
+class sd_unet_cfg(ctypes.Structure):
+    _fields_ = [("in_channels", c_int32), ("out_channels", c_int32), ("height", c_int32), ("width", c_int32),
+                ("n_levels", c_int32), ("block_channels", c_int32 * 4), ("attn_depth", c_int32 * 4),
+                ("layers_per_block", c_int32), ("mid_depth", c_int32), ("head_dim", c_int32),
+                ("ctx_len", c_int32), ("ctx_dim", c_int32), ("time_proj_dim", c_int32), ("temb_dim", c_int32),
+                ("groups", c_int32), ("eps", c_float)]
+
+
+# name -> (restype, argtypes)
+_P = c_void_p
+_SIGS = {
+    "sd_version": (c_char_p, []),
+    "sd_status_string": (c_char_p, [c_int32]),
+    "sd_time_weight_layout": (c_int32, [POINTER(sd_time_cfg), POINTER(sd_tensor_desc), c_int32, POINTER(c_int32),
+                                        POINTER(c_int64), POINTER(c_int64)]),
+    "sd_conv_weight_layout": (c_int32, [POINTER(sd_conv_cfg), c_int32, POINTER(sd_tensor_desc), c_int32,
+                                        POINTER(c_int32), POINTER(c_int64), POINTER(c_int64)]),
+    "sd_resblock_weight_layout": (c_int32, [POINTER(sd_resblock_cfg), POINTER(sd_tensor_desc), c_int32,
+                                            POINTER(c_int32), POINTER(c_int64), POINTER(c_int64)]),
+    "sd_transformer_weight_layout": (c_int32, [POINTER(sd_transformer_cfg), POINTER(sd_tensor_desc), c_int32,
+                                               POINTER(c_int32), POINTER(c_int64), POINTER(c_int64)]),
+    "sd_unet_weight_layout": (c_int32, [POINTER(sd_unet_cfg), POINTER(sd_tensor_desc), c_int32, POINTER(c_int32),
+                                        POINTER(c_int64), POINTER(c_int64)]),
+    "sd_time_pack_weights": (c_int32, [POINTER(sd_time_cfg), POINTER(c_uint16), _P]),
+    "sd_conv_pack_weights": (c_int32, [POINTER(sd_conv_cfg), c_int32, POINTER(c_uint16), _P]),
+    "sd_resblock_pack_weights": (c_int32, [POINTER(sd_resblock_cfg), POINTER(c_uint16), _P]),
+    "sd_transformer_pack_weights": (c_int32, [POINTER(sd_transformer_cfg), POINTER(c_uint16), _P]),
+    "sd_unet_pack_weights": (c_int32, [POINTER(sd_unet_cfg), POINTER(c_uint16), _P]),
+    "sd_time_workspace_size": (c_size_t, [POINTER(sd_time_cfg)]),
+    "sd_conv_workspace_size": (c_size_t, [POINTER(sd_conv_cfg), c_int32]),
+    "sd_resblock_workspace_size": (c_size_t, [POINTER(sd_resblock_cfg)]),
+    "sd_transformer_workspace_size": (c_size_t, [POINTER(sd_transformer_cfg)]),
+    "sd_unet_workspace_size": (c_size_t, [POINTER(sd_unet_cfg)]),
+    "sd_time_embed": (c_int32, [POINTER(sd_time_cfg), _P, c_float, _P, _P, c_size_t, _P]),
+    "sd_conv_fwd": (c_int32, [POINTER(sd_conv_cfg), c_int32, _P, _P, _P, _P, _P, _P, c_size_t, _P]),
+    "sd_resblock_fwd": (c_int32, [POINTER(sd_resblock_cfg), _P, _P, _P, _P, _P, _P, c_size_t, _P]),
+    "sd_transformer_fwd": (c_int32, [POINTER(sd_transformer_cfg), _P, _P, _P, _P, _P, c_size_t, _P]),
+    "sd_unet_step": (c_int32, [POINTER(sd_unet_cfg), _P, _P, c_float, _P, _P, _P, c_size_t, _P]),
+    "sd_query_device_status": (c_int32, [_P, _P]),
+}
+
+_lib = None
+
+
+def lib():
+    """Load the shared library (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                               "(run python -m latent_diffusion_net_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def status_string(s: int) -> str:
+    try:
+        return lib().sd_status_string(int(s)).decode()
+    except Exception:  # noqa: BLE001 - used while formatting another error
+        return "?"
+
+
+def _check(status: int, where: str):
+    if status != SD_OK:
+        raise SdError(status, where)
+    return status
+
+
+def _ptr(x):
+    """Device or host address of a torch tensor, an int, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ---------------------------------------------------------------- tables and packing
+
+def _table(fn, *args):
+    n = c_int32(0)
+    ce = c_int64(0)
+    pb = c_int64(0)
+    _check(fn(*args, None, 0, ctypes.byref(n), ctypes.byref(ce), ctypes.byref(pb)), fn.__name__)
+    arr = (sd_tensor_desc * n.value)()
+    _check(fn(*args, arr, n.value, ctypes.byref(n), ctypes.byref(ce), ctypes.byref(pb)), fn.__name__)
+    rows = []
+    for d in arr:
+        rows.append({"name": d.name.decode(), "shape": tuple(d.shape[i] for i in range(d.ndim)),
+                     "kind": KIND_NAMES[d.kind], "fan_in": d.fan_in, "canon_offset": d.canon_offset,
+                     "packed_offset": d.packed_offset})
+    return rows, ce.value, pb.value
+
+
+def sd_time_weight_layout(cfg):
+    return _table(lib().sd_time_weight_layout, ctypes.byref(cfg))
+
+
+def sd_conv_weight_layout(cfg, kind):
+    return _table(lib().sd_conv_weight_layout, ctypes.byref(cfg), int(kind))
+
+
+def sd_resblock_weight_layout(cfg):
+    return _table(lib().sd_resblock_weight_layout, ctypes.byref(cfg))
+
+
+def sd_transformer_weight_layout(cfg):
+    return _table(lib().sd_transformer_weight_layout, ctypes.byref(cfg))
+
+
+def sd_unet_weight_layout(cfg):
+    return _table(lib().sd_unet_weight_layout, ctypes.byref(cfg))
+
+
+def _pack(fn, args, canonical_u16, packed_bytes):
+    import numpy as np
+    canon = np.ascontiguousarray(canonical_u16, dtype=np.uint16)
+    out = np.empty(packed_bytes, dtype=np.uint8)
+    _check(fn(*args, canon.ctypes.data_as(POINTER(c_uint16)), out.ctypes.data_as(c_void_p)), fn.__name__)
+    return out
+
+
+def sd_time_pack_weights(cfg, canonical_u16, packed_bytes):
+    return _pack(lib().sd_time_pack_weights, (ctypes.byref(cfg),), canonical_u16, packed_bytes)
+
+
+def sd_conv_pack_weights(cfg, kind, canonical_u16, packed_bytes):
+    return _pack(lib().sd_conv_pack_weights, (ctypes.byref(cfg), int(kind)), canonical_u16, packed_bytes)
+
+
+def sd_resblock_pack_weights(cfg, canonical_u16, packed_bytes):
+    return _pack(lib().sd_resblock_pack_weights, (ctypes.byref(cfg),), canonical_u16, packed_bytes)
+
+
+def sd_transformer_pack_weights(cfg, canonical_u16, packed_bytes):
+    return _pack(lib().sd_transformer_pack_weights, (ctypes.byref(cfg),), canonical_u16, packed_bytes)
+
+
+def sd_unet_pack_weights(cfg, canonical_u16, packed_bytes):
+    return _pack(lib().sd_unet_pack_weights, (ctypes.byref(cfg),), canonical_u16, packed_bytes)
+
+
+# ---------------------------------------------------------------- workspace sizes
+
+def sd_time_workspace_size(cfg):
+    return lib().sd_time_workspace_size(ctypes.byref(cfg))
+
+
+def sd_conv_workspace_size(cfg, kind):
+    return lib().sd_conv_workspace_size(ctypes.byref(cfg), int(kind))
+
+
+def sd_resblock_workspace_size(cfg):
+    return lib().sd_resblock_workspace_size(ctypes.byref(cfg))
+
+
+def sd_transformer_workspace_size(cfg):
+    return lib().sd_transformer_workspace_size(ctypes.byref(cfg))
+
+
+def sd_unet_workspace_size(cfg):
+    return lib().sd_unet_workspace_size(ctypes.byref(cfg))
+
+
+# ---------------------------------------------------------------- forward calls
+# Each returns the status (SD_OK) or raises SdError; pass check=False to get
+# the raw status instead.
+
+def sd_time_embed(cfg, packed_w, timestep, temb_out, workspace, ws_bytes, stream=None, check=True):
+    s = lib().sd_time_embed(ctypes.byref(cfg), _ptr(packed_w), float(timestep), _ptr(temb_out), _ptr(workspace),
+                            int(ws_bytes), _stream(stream))
+    return _check(s, "sd_time_embed") if check else s
+
+
+def sd_conv_fwd(cfg, kind, packed_w, x0, x1, x2, y, workspace, ws_bytes, stream=None, check=True):
+    s = lib().sd_conv_fwd(ctypes.byref(cfg), int(kind), _ptr(packed_w), _ptr(x0), _ptr(x1), _ptr(x2), _ptr(y),
+                          _ptr(workspace), int(ws_bytes), _stream(stream))
+    return _check(s, "sd_conv_fwd") if check else s
+
+
+def sd_resblock_fwd(cfg, packed_w, x, skip, temb, y, workspace, ws_bytes, stream=None, check=True):
+    s = lib().sd_resblock_fwd(ctypes.byref(cfg), _ptr(packed_w), _ptr(x), _ptr(skip), _ptr(temb), _ptr(y),
+                              _ptr(workspace), int(ws_bytes), _stream(stream))
+    return _check(s, "sd_resblock_fwd") if check else s
+
+
+def sd_transformer_fwd(cfg, packed_w, x, context, y, workspace, ws_bytes, stream=None, check=True):
+    s = lib().sd_transformer_fwd(ctypes.byref(cfg), _ptr(packed_w), _ptr(x), _ptr(context), _ptr(y),
+                                 _ptr(workspace), int(ws_bytes), _stream(stream))
+    return _check(s, "sd_transformer_fwd") if check else s
+
+
+def sd_unet_step(cfg, packed_w, latent, timestep, context, eps_out, workspace, ws_bytes, stream=None, check=True):
+    s = lib().sd_unet_step(ctypes.byref(cfg), _ptr(packed_w), _ptr(latent), float(timestep), _ptr(context),
+                           _ptr(eps_out), _ptr(workspace), int(ws_bytes), _stream(stream))
+    return _check(s, "sd_unet_step") if check else s
+
+
+def sd_query_device_status(workspace, stream=None):
+    return lib().sd_query_device_status(_ptr(workspace), _stream(stream))
+
+
+# ---------------------------------------------------------------- config helpers
+
+def time_cfg(proj_dim=320, temb_dim=1280):
+    return sd_time_cfg(proj_dim, temb_dim)
+
+
+def conv_cfg(height, width, c_in, c_out, groups=32, eps=1e-5):
+    return sd_conv_cfg(1, height, width, c_in, c_out, groups, eps)
+
+
+def resblock_cfg(height, width, c_x, c_out, c_skip=0, temb_dim=1280, groups=32, eps=1e-5):
+    return sd_resblock_cfg(1, height, width, c_x, c_skip, c_out, temb_dim, groups, eps)
+
+
+def transformer_cfg(height, width, channels, depth=1, ctx_len=77, ctx_dim=1024, groups=32, eps=1e-5):
+    return sd_transformer_cfg(1, height, width, channels, 64, depth, ctx_len, ctx_dim, groups, eps, eps)
+
+
+def unet_cfg(in_channels=4, out_channels=4, height=96, width=96, block_channels=(320, 640, 1280, 1280),
+             attn_depth=(1, 1, 1, 0), layers_per_block=2, mid_depth=1, ctx_len=77, ctx_dim=1024,
+             time_proj_dim=320, temb_dim=1280, groups=32, eps=1e-5):
+    bc = list(block_channels) + [0] * (4 - len(block_channels))
+    ad = list(attn_depth) + [0] * (4 - len(attn_depth))
+    return sd_unet_cfg(in_channels, out_channels, height, width, len(block_channels), (c_int32 * 4)(*bc),
+                       (c_int32 * 4)(*ad), layers_per_block, mid_depth, 64, ctx_len, ctx_dim, time_proj_dim,
+                       temb_dim, groups, eps)

@@ -1,0 +1,73 @@
+// Host-visible description of the tcgen05 implicit-GEMM used for every dense
+// contraction of the denoiser: 3x3 convolutions (9 shifted K-segments over an
+// NHWC activation), stride-2 convolutions (9 segments over 4 phase planes),
+// 1x1 shortcut convolutions fused as extra K-segments, and token linears.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sdk {
+
+constexpr int kGemmMaxSeg = 12;
+constexpr int kGemmMaxA = 4;
+constexpr int kGemmMaxB = 2;
+
+enum GemmMode : int32_t { GEMM_PLAIN = 0, GEMM_GEGLU = 1 };
+
+// One activation source: a BF16 NHWC tensor seen as [Z][H][W][C].
+struct GemmASrc {
+  const void* ptr;
+  int32_t C, W, H, Z;
+};
+
+// One weight matrix: BF16 [rows][K] row-major (rows = output features).
+struct GemmBSrc {
+  const void* ptr;
+  int32_t K, rows;
+};
+
+// K-segment: nkb blocks of 64 reduction elements read from A source `amap` at
+// channel c0 with the output tile shifted by (dx, dy) on plane z, against B
+// source `bmap` starting at reduction index bk0.
+struct GemmSeg {
+  int32_t amap, bmap;
+  int32_t dx, dy, z;
+  int32_t c0, bk0, nkb;
+};
+
+struct GemmEpi {
+  const __nv_bfloat16* bias;      // [N] or null
+  const __nv_bfloat16* bias2;     // [N] or null (second bias, e.g. a fused shortcut)
+  const float* colvec;            // [N] FP32 or null (time-embedding projection)
+  const __nv_bfloat16* residual;  // [M][ld_res] or null, added after the biases
+  int32_t ld_res;
+  __nv_bfloat16* out;             // [M][ld_out]
+  int32_t ld_out;
+  int32_t mode;                   // GemmMode
+};
+
+// A full problem: output grid Ho x Wo (M = Ho*Wo rows), N output features.
+struct GemmProblem {
+  int32_t Ho, Wo, N;
+  int32_t na, nb, nseg;
+  GemmASrc a[kGemmMaxA];
+  GemmBSrc b[kGemmMaxB];
+  GemmSeg seg[kGemmMaxSeg];
+  GemmEpi epi;
+  int* err;
+  int32_t force_bn;  // 0 = heuristic
+};
+
+// Launch on `stream`. Returns 0 on success, a cudaError_t value otherwise
+// (or -1 for an unsupported shape).
+int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream);
+
+// Tensor-map encoder from the driver (resolved once, no -lcuda needed).
+bool tmap_encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                    uint32_t box_outer);
+bool tmap_encode_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4], uint32_t box_w, uint32_t box_h);
+
+}  // namespace sdk

@@ -1,0 +1,58 @@
+// Launchers of the non-GEMM kernels. Each returns 0 or a cudaError_t value.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sdk {
+
+// GroupNorm: statistics over the channel concatenation [x0 | x1] (x1 may be
+// null with C1 = 0); `partial` holds gn_stats_blocks() * G float2 values and
+// `counter` one zero-initialised word (left at zero on return).
+int gn_stats_blocks(int HW, int C, int num_sms);
+int launch_gn_stats(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G, float eps,
+                    float2* partial, unsigned int* counter, float2* stats, int num_sms, cudaStream_t st);
+int launch_gn_apply(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G,
+                    const float2* stats, const __nv_bfloat16* gamma, const __nv_bfloat16* beta, int silu,
+                    __nv_bfloat16* y, int num_sms, cudaStream_t st);
+int launch_layernorm(const __nv_bfloat16* x, int N, int C, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,
+                     float eps, __nv_bfloat16* y, cudaStream_t st);
+
+// Time embedding: phi(t) sinusoid [proj_dim] into out (FP32).
+int launch_sinusoid(float t, int proj_dim, float* out, cudaStream_t st);
+
+// Grouped GEMV: for each job, y[r] = act_out(sum_k W[r][k] * act_in(x[k]) + b[r]),
+// W BF16 [rows][K] row-major, x FP32 [K] shared by all jobs.
+constexpr int kMaxGemvJobs = 32;
+struct GemvJob {
+  const __nv_bfloat16* W;
+  const __nv_bfloat16* b;
+  float* y;
+  int32_t rows;
+};
+struct GemvBatch {
+  int32_t njobs, K, silu_in, silu_out;
+  const float* x;
+  GemvJob job[kMaxGemvJobs];
+};
+int launch_gemv(const GemvBatch& batch, cudaStream_t st);
+
+// Nearest 2x upsample of NHWC [H, W, C] into [2H, 2W, C].
+int launch_upsample2x(const __nv_bfloat16* x, int H, int W, int C, __nv_bfloat16* y, cudaStream_t st);
+
+// Phase split for the stride-2 convolution: y[a*2+b][i][j][c] = x[2i+a][2j+b][c].
+int launch_phase_split(const __nv_bfloat16* x, int H, int W, int C, __nv_bfloat16* y, cudaStream_t st);
+
+// conv_in operand: y[p][k] for k = (ky*3 + kx)*Cin + c (0 beyond 9*Cin, up to Kp),
+// reading input channel c from the source that holds it (up to 3 sources of
+// widths c0/c1/c2 concatenated on channels), zero outside the image.
+int launch_conv_in_im2col(const __nv_bfloat16* s0, int c0, const __nv_bfloat16* s1, int c1,
+                          const __nv_bfloat16* s2, int c2, int H, int W, int Kp, __nv_bfloat16* y,
+                          cudaStream_t st);
+
+// Flash attention (head_dim 64): O[i, h*64 + d] = softmax_j(Q_i.K_j / 8) V_j per head.
+int launch_attention(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk, const __nv_bfloat16* V,
+                     int ldv, __nv_bfloat16* O, int ldo, int Nq, int Nk, int heads, cudaStream_t st);
+
+}  // namespace sdk

@@ -1,0 +1,112 @@
+// Weight tables: the canonical tensor list of every module (names, shapes,
+// kinds, fan-in) and the packed layout the kernels read. Pure host code.
+#pragma once
+
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "sd_api.h"
+
+namespace sdw {
+
+enum Pack : int {
+  PACK_COPY = 0,     // same element order
+  PACK_CONV_KRSC,    // [O][C][kh][kw] -> [O][kh][kw][C]
+  PACK_CONV_IM2COL,  // [O][C][3][3]  -> [O][Kp], k = (ky*3+kx)*C + c, zero-padded to Kp
+  PACK_GEGLU_ROWS,   // [8C][C]: row 2j = value row j, row 2j+1 = gate row 4C + j
+  PACK_GEGLU_BIAS    // [8C]: same interleave
+};
+
+struct Tensor {
+  std::string name;
+  int ndim = 0;
+  int64_t shape[4] = {0, 0, 0, 0};
+  int kind = 0;
+  int fan_in = 0;
+  int64_t canon_off = 0;   // elements
+  int64_t packed_off = 0;  // bytes
+  int pack = PACK_COPY;
+  int64_t packed_elems = 0;
+  int aux = 0;  // PACK_CONV_IM2COL: Kp
+  int64_t numel() const {
+    int64_t n = 1;
+    for (int i = 0; i < ndim; ++i) n *= shape[i];
+    return n;
+  }
+};
+
+struct Table {
+  std::vector<Tensor> t;
+  int64_t canon_elems = 0;
+  int64_t packed_bytes = 0;
+  // Appends a tensor; returns its packed byte offset.
+  int64_t add(const std::string& name, std::initializer_list<int64_t> shape, int kind, int fan_in,
+              int pack = PACK_COPY, int aux = 0);
+};
+
+// Packed byte offsets of each module's tensors.
+struct TimeW {
+  int64_t l1w, l1b, l2w, l2b;
+};
+struct ConvW {
+  int64_t w, b;
+};
+struct OutW {
+  int64_t ng, nb, w, b;
+};
+struct ResW {
+  int c_in, c_out;
+  int64_t n1g, n1b, c1w, c1b, tw, tb, n2g, n2b, c2w, c2b, sw, sb;  // sw/sb = -1 without shortcut
+};
+struct TxBlockW {
+  int64_t ln1g, ln1b, qkv, o1w, o1b, ln2g, ln2b, q2, kv2, o2w, o2b, ln3g, ln3b, f1w, f1b, f2w, f2b;
+};
+struct TxW {
+  int C, depth, ctx_dim;
+  int64_t ng, nb, piw, pib, pow_, pob;
+  std::vector<TxBlockW> blocks;
+};
+
+TimeW add_time(Table& tab, const std::string& prefix, int proj_dim, int temb_dim);
+ConvW add_conv3x3(Table& tab, const std::string& prefix, int c_in, int c_out);
+ConvW add_conv_in(Table& tab, const std::string& prefix, int c_in, int c_out, int kp);
+OutW add_output(Table& tab, int c_in, int c_out);
+ResW add_resblock(Table& tab, const std::string& prefix, int c_in, int c_out, int temb_dim);
+TxW add_transformer(Table& tab, const std::string& prefix, int C, int depth, int ctx_dim);
+
+// Whole U-Net: module order follows the forward pass.
+struct UNetW {
+  TimeW time;
+  ConvW conv_in;
+  int conv_in_kp;
+  struct Level {
+    std::vector<ResW> res;
+    std::vector<TxW> attn;  // empty when the level has no attention
+    bool has_down;
+    ConvW down;
+  };
+  std::vector<Level> down;
+  ResW mid_res0, mid_res1;
+  TxW mid_attn;
+  struct UpLevel {
+    std::vector<ResW> res;
+    std::vector<TxW> attn;
+    bool has_up;
+    ConvW up;
+  };
+  std::vector<UpLevel> up;
+  OutW out;
+};
+UNetW add_unet(Table& tab, const sd_unet_cfg& cfg);
+
+int conv_in_kp(int c_in);
+
+// Canonical (host, BF16 bits) -> packed (host).
+void pack(const Table& tab, const uint16_t* canonical, uint8_t* packed);
+
+sd_status export_table(const Table& tab, sd_tensor_desc* out, int32_t capacity, int32_t* n_tensors,
+                       int64_t* canon_elems, int64_t* packed_bytes);
+
+}  // namespace sdw

@@ -152,3 +152,18 @@ def param_value(seed: int, k: int, shape, kind: str, fan_in: int, affine_noise: 
             return normal_bf16(seed, idx, shape, 0.1)
         return np.zeros(shape, dtype=np.float32)
     raise ValueError(kind)
+
+
+def canonical_weights(rows, seed: int, affine_noise: bool = False, index_base: int = 0) -> np.ndarray:
+    """Canonical BF16 buffer (uint16 bit patterns) for a weight table.
+
+    ``rows`` is a sequence of (shape, kind, fan_in) in table order; tensor ``i``
+    uses generator stream ``WEIGHT_INDEX_BASE + index_base + i``."""
+    sizes = [int(np.prod(s)) for s, _, _ in rows]
+    out = np.empty(sum(sizes), dtype=np.uint16)
+    off = 0
+    for i, ((shape, kind, fan), n) in enumerate(zip(rows, sizes)):
+        v = param_value(seed, index_base + i, tuple(shape), kind, fan, affine_noise)
+        out[off:off + n] = f32_to_bf16_bits(np.ascontiguousarray(v, dtype=np.float32).reshape(-1))
+        off += n
+    return out

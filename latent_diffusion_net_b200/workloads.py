@@ -1,0 +1,31 @@
+"""The five synthetic workloads (shapes, seeds, value distributions).
+
+Every input is N(0, 1) rounded to BF16; every convolution/linear weight and
+bias is N(0, 1/fan_in) rounded to BF16; norm gains are 1 and shifts 0; the
+timestep is 500. Activations are NHWC.
+
+1. crossattn_block_320x32: time MLP + ResnetBlock2D 320->320 + Transformer2DModel
+   depth 1 (5 heads x 64) at 32x32, context [77, 1024]; seed 0.
+2. crossattn_block_320x96: the same block at the SD2.1-base level-0 size 96x96
+   (9216 tokens); seed 1.
+3. sdxl_level1_stage_640x64: time MLP + 2 x (ResnetBlock2D 640 + Transformer2DModel
+   depth 2, 10 heads) at 64x64, context [77, 2048], then a stride-2 downsample;
+   seed 2.
+4. sdxl_level2_stage_1280x32: time MLP + ResnetBlock2D 1280 + Transformer2DModel
+   depth 10 (20 heads) at 32x32, context [77, 2048]; plus the inpaint conv_in
+   9->320 on a 128x128 input assembled from a noisy latent, a masked latent and a
+   rectangle mask; seed 3.
+5. sd21_base_unet_step_96: the whole SD2.1-base-shaped denoiser step on a 96x96
+   latent with 4 channels, context [77, 1024]; seed 4.
+"""
+
+WORKLOADS = {
+    1: dict(name="crossattn_block_320x32", seed=0, kind="block", H=32, W=32, C=320, depth=1, ctx_dim=1024),
+    2: dict(name="crossattn_block_320x96", seed=1, kind="block", H=96, W=96, C=320, depth=1, ctx_dim=1024),
+    3: dict(name="sdxl_level1_stage_640x64", seed=2, kind="stage3", H=64, W=64, C=640, depth=2, ctx_dim=2048),
+    4: dict(name="sdxl_level2_stage_1280x32", seed=3, kind="stage4", H=32, W=32, C=1280, depth=10, ctx_dim=2048,
+            inpaint_hw=128),
+    5: dict(name="sd21_base_unet_step_96", seed=4, kind="unet", H=96, W=96, ctx_dim=1024),
+}
+TIMESTEP = 500.0
+CTX_LEN = 77
