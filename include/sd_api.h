@@ -218,7 +218,8 @@ sd_status sd_resblock_fwd(const sd_resblock_cfg* cfg, const void* packed_w, cons
                           const void* skip, const float* temb, void* y, void* workspace, size_t ws_bytes,
                           sd_stream_t stream);
 
-/* x [H, W, C], context [ctx_len, ctx_dim], y [H, W, C]. */
+/* x [H, W, C], context [ctx_len, ctx_dim], y [H, W, C]; y may alias x (in-place
+ * update of the residual stream). */
 sd_status sd_transformer_fwd(const sd_transformer_cfg* cfg, const void* packed_w, const void* x,
                              const void* context, void* y, void* workspace, size_t ws_bytes,
                              sd_stream_t stream);
@@ -235,6 +236,37 @@ sd_status sd_unet_step(const sd_unet_cfg* cfg, const void* packed_w, const void*
  * SD_OK, or SD_ERR_DEVICE_TIMEOUT when a bounded wait gave up; the word is
  * cleared afterwards. */
 sd_status sd_query_device_status(void* workspace, sd_stream_t stream);
+
+/* ---------------------------------------------------------------- launch accounting
+ * Optional per-thread recorder for measuring kernels in place: between
+ * sd_profile_begin() and sd_profile_end() every kernel this library launches
+ * from the calling thread is bracketed by two CUDA events on its stream and
+ * tagged with its algorithmic FLOPs (2*M*N*K per contraction, 4*Nq*Nk*C per
+ * attention) and bytes (each operand read once, each output written once).
+ * Recording also works while the stream is being captured into a CUDA graph,
+ * provided an earlier eager recording of the same call sequence created the
+ * events; the graph then holds the event records and every replay overwrites
+ * them. sd_profile_read() returns the records of the last recording with their
+ * elapsed times (ms < 0 where the events have not completed). */
+typedef struct {
+  char kernel[24];  /* "gemm_tc", "attention", "gn_stats", "gn_apply", "layernorm", "gemv", ... */
+  int32_t family;   /* SD_FAMILY_* */
+  double flops;
+  double bytes;
+  float ms;
+} sd_launch_record;
+
+enum {
+  SD_FAMILY_GEMM = 0, SD_FAMILY_ATTENTION = 1, SD_FAMILY_GN_STATS = 2, SD_FAMILY_GN_APPLY = 3,
+  SD_FAMILY_LAYERNORM = 4, SD_FAMILY_GEMV = 5, SD_FAMILY_OTHER = 6
+};
+
+sd_status sd_profile_begin(void);
+sd_status sd_profile_end(int32_t* n_launches);
+sd_status sd_profile_read(sd_launch_record* out, int32_t capacity, int32_t* n);
+
+/* Kernel launches issued by this library in this process so far. */
+int64_t sd_launch_count(void);
 
 const char* sd_status_string(sd_status s);
 

@@ -63,6 +63,13 @@ class sd_unet_cfg(ctypes.Structure):
                 ("groups", c_int32), ("eps", c_float)]
 
 
+class sd_launch_record(ctypes.Structure):
+    _fields_ = [("kernel", c_char * 24), ("family", c_int32), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double), ("ms", c_float)]
+
+
+FAMILY_NAMES = {0: "gemm_tc", 1: "attention", 2: "gn_stats", 3: "gn_apply", 4: "layernorm", 5: "gemv", 6: "other"}
+
 # name -> (restype, argtypes)
 _P = c_void_p
 _SIGS = {
@@ -94,6 +101,10 @@ _SIGS = {
     "sd_transformer_fwd": (c_int32, [POINTER(sd_transformer_cfg), _P, _P, _P, _P, _P, c_size_t, _P]),
     "sd_unet_step": (c_int32, [POINTER(sd_unet_cfg), _P, _P, c_float, _P, _P, _P, c_size_t, _P]),
     "sd_query_device_status": (c_int32, [_P, _P]),
+    "sd_profile_begin": (c_int32, []),
+    "sd_profile_end": (c_int32, [POINTER(c_int32)]),
+    "sd_profile_read": (c_int32, [POINTER(sd_launch_record), c_int32, POINTER(c_int32)]),
+    "sd_launch_count": (c_int64, []),
 }
 
 _lib = None
@@ -272,6 +283,30 @@ def sd_unet_step(cfg, packed_w, latent, timestep, context, eps_out, workspace, w
 
 def sd_query_device_status(workspace, stream=None):
     return lib().sd_query_device_status(_ptr(workspace), _stream(stream))
+
+
+def sd_profile_begin():
+    return _check(lib().sd_profile_begin(), "sd_profile_begin")
+
+
+def sd_profile_end():
+    n = c_int32(0)
+    _check(lib().sd_profile_end(ctypes.byref(n)), "sd_profile_end")
+    return n.value
+
+
+def sd_profile_read():
+    """Records of the last recording: list of dicts (kernel, family, flops, bytes, ms)."""
+    n = c_int32(0)
+    _check(lib().sd_profile_read(None, 0, ctypes.byref(n)), "sd_profile_read")
+    arr = (sd_launch_record * max(n.value, 1))()
+    _check(lib().sd_profile_read(arr, n.value, ctypes.byref(n)), "sd_profile_read")
+    return [{"kernel": r.kernel.decode(), "family": FAMILY_NAMES.get(r.family, r.family), "flops": r.flops,
+             "bytes": r.bytes, "ms": r.ms} for r in arr[:n.value]]
+
+
+def sd_launch_count():
+    return int(lib().sd_launch_count())
 
 
 # ---------------------------------------------------------------- config helpers

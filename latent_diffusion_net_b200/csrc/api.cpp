@@ -13,6 +13,7 @@
 
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
+#include "profile.h"
 #include "sd_api.h"
 #include "weights.h"
 
@@ -102,12 +103,44 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 // ------------------------------------------------------------------ building blocks
 
+int run_gemv(const Ctx& c, const sdk::GemvBatch& b) {
+  double rows = 0;
+  for (int j = 0; j < b.njobs; ++j) rows += b.job[j].rows;
+  sdp::Scope sc("gemv", sdp::F_GEMV, 2.0 * rows * b.K, 2.0 * rows * b.K, c.st);
+  return sdk::launch_gemv(b, c.st);
+}
+
 // GroupNorm (+SiLU) of [x0 | x1] into y.
 sd_status run_gn(const Ctx& c, const bf16* x0, int C0, const bf16* x1, int C1, int HW, int G, float eps,
                  const bf16* gamma, const bf16* beta, int silu, bf16* y) {
-  CK(sdk::launch_gn_stats(x0, C0, x1, C1, HW, G, eps, c.partial, c.counter, c.stats, c.sms, c.st));
-  CK(sdk::launch_gn_apply(x0, C0, x1, C1, HW, G, c.stats, gamma, beta, silu, y, c.sms, c.st));
+  const double bytes = (double)HW * (C0 + C1) * 2;
+  {
+    sdp::Scope sc("gn_stats", sdp::F_GN_STATS, 0, bytes, c.st);
+    CK(sdk::launch_gn_stats(x0, C0, x1, C1, HW, G, eps, c.partial, c.counter, c.stats, c.sms, c.st));
+  }
+  {
+    sdp::Scope sc("gn_apply", sdp::F_GN_APPLY, 0, 2 * bytes, c.st);
+    CK(sdk::launch_gn_apply(x0, C0, x1, C1, HW, G, c.stats, gamma, beta, silu, y, c.sms, c.st));
+  }
   return SD_OK;
+}
+
+// Launch a GEMM problem under a profiling scope with its algorithmic work:
+// FLOPs 2*M*N*K (K = reduction length; alg_k overrides a zero-padded K), bytes
+// = every A source and B matrix read once, the output (and residual) once.
+int launch_gemm(const Ctx& c, const GemmProblem& p, double alg_k = 0) {
+  double K = 0;
+  for (int i = 0; i < p.nseg; ++i) K += 64.0 * p.seg[i].nkb;
+  if (alg_k > 0) K = alg_k;
+  const double M = (double)p.Ho * p.Wo;
+  const double fl = 2.0 * M * p.N * K;
+  double by = 0;
+  for (int i = 0; i < p.na; ++i) by += 2.0 * p.a[i].C * p.a[i].W * p.a[i].H * p.a[i].Z;
+  for (int i = 0; i < p.nb; ++i) by += 2.0 * p.b[i].K * (p.b[i].rows < p.N ? p.b[i].rows : p.N);
+  by += 2.0 * M * (p.epi.mode == sdk::GEMM_GEGLU ? p.N / 2 : p.N);
+  if (p.epi.residual) by += 2.0 * M * p.N;
+  sdp::Scope sc("gemm_tc", sdp::F_GEMM, fl, by, c.st);
+  return sdk::gemm_tc_launch(p, c.st);
 }
 
 GemmProblem base_problem(const Ctx& c) {
@@ -133,7 +166,8 @@ void add_conv3x3_segs(GemmProblem& p, int amap, int bmap, int C) {
 
 // y[M, N] = A[M, K] B[N, K]^T (+ epilogue), A a token matrix.
 sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, int N, const bf16* bias,
-                     const bf16* residual, int ld_res, bf16* out, int ld_out, int mode = sdk::GEMM_PLAIN) {
+                     const bf16* residual, int ld_res, bf16* out, int ld_out, int mode = sdk::GEMM_PLAIN,
+                     double alg_k = 0) {
   GemmProblem p = base_problem(c);
   p.Ho = 1;
   p.Wo = M;
@@ -150,7 +184,7 @@ sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, i
   p.epi.out = out;
   p.epi.ld_out = ld_out;
   p.epi.mode = mode;
-  CK(sdk::gemm_tc_launch(p, c.st));
+  CK(launch_gemm(c, p, alg_k));
   return SD_OK;
 }
 
@@ -169,7 +203,7 @@ sd_status run_conv3x3(const Ctx& c, const bf16* x, int H, int Wd, int C, const b
   p.epi.bias = bias;
   p.epi.out = out;
   p.epi.ld_out = N;
-  CK(sdk::gemm_tc_launch(p, c.st));
+  CK(launch_gemm(c, p));
   return SD_OK;
 }
 
@@ -208,7 +242,7 @@ sd_status run_resblock(const Ctx& c, const ResW& w, const void* pw, int H, int W
     p.epi.colvec = tproj;
     p.epi.out = s.h1;
     p.epi.ld_out = cout;
-    CK(sdk::gemm_tc_launch(p, c.st));
+    CK(launch_gemm(c, p));
   }
   // y = conv2(SiLU(GN2(h1))) + b2 + shortcut
   if ((r = run_gn(c, s.h1, cout, nullptr, 0, HW, G, eps, W(pw, w.n2g), W(pw, w.n2b), 1, s.hn)) != SD_OK) return r;
@@ -242,7 +276,7 @@ sd_status run_resblock(const Ctx& c, const ResW& w, const void* pw, int H, int W
       p.epi.residual = x;
       p.epi.ld_res = cout;
     }
-    CK(sdk::gemm_tc_launch(p, c.st));
+    CK(launch_gemm(c, p));
   }
   return SD_OK;
 }
@@ -260,6 +294,18 @@ TxScratch plan_tx_scratch(Arena& ar, int HW, int C, int ctx_len) {
   return s;
 }
 
+int run_ln(const Ctx& c, const bf16* x, int N, int C, const bf16* g, const bf16* b, float eps, bf16* y) {
+  sdp::Scope sc("layernorm", sdp::F_LN, 0, 4.0 * N * C, c.st);
+  return sdk::launch_layernorm(x, N, C, g, b, eps, y, c.st);
+}
+
+int run_attn(const Ctx& c, const bf16* q, int ldq, const bf16* k, int ldk, const bf16* v, int ldv, bf16* o, int ldo,
+             int Nq, int Nk, int heads) {
+  const double C = 64.0 * heads;
+  sdp::Scope sc("attention", sdp::F_ATTN, 4.0 * Nq * Nk * C, 2.0 * C * (2.0 * Nq + 2.0 * Nk), c.st);
+  return sdk::launch_attention(q, ldq, k, ldk, v, ldv, o, ldo, Nq, Nk, heads, c.st);
+}
+
 // Transformer2DModel; y may alias x.
 sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int Wd, const bf16* x, const bf16* ctx,
                           int ctx_len, int G, float gn_eps, float ln_eps, bf16* y, const TxScratch& s) {
@@ -271,19 +317,19 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
   if ((r = run_linear(c, s.nrm, HW, C, W(pw, w.piw), C, W(pw, w.pib), nullptr, 0, s.t, C)) != SD_OK) return r;
   for (const TxBlockW& b : w.blocks) {
     // self-attention: t += Wo Attn(LN1(t))
-    CK(sdk::launch_layernorm(s.t, HW, C, W(pw, b.ln1g), W(pw, b.ln1b), ln_eps, s.nrm, c.st));
+    CK(run_ln(c, s.t, HW, C, W(pw, b.ln1g), W(pw, b.ln1b), ln_eps, s.nrm));
     if ((r = run_linear(c, s.nrm, HW, C, W(pw, b.qkv), 3 * C, nullptr, nullptr, 0, s.big, 3 * C)) != SD_OK) return r;
-    CK(sdk::launch_attention(s.big, 3 * C, s.big + C, 3 * C, s.big + 2 * C, 3 * C, s.ao, C, HW, HW, heads, c.st));
+    CK(run_attn(c, s.big, 3 * C, s.big + C, 3 * C, s.big + 2 * C, 3 * C, s.ao, C, HW, HW, heads));
     if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o1w), C, W(pw, b.o1b), s.t, C, s.t, C)) != SD_OK) return r;
     // cross-attention: t += Wo' Attn(LN2(t), ctx)
-    CK(sdk::launch_layernorm(s.t, HW, C, W(pw, b.ln2g), W(pw, b.ln2b), ln_eps, s.nrm, c.st));
+    CK(run_ln(c, s.t, HW, C, W(pw, b.ln2g), W(pw, b.ln2b), ln_eps, s.nrm));
     if ((r = run_linear(c, s.nrm, HW, C, W(pw, b.q2), C, nullptr, nullptr, 0, s.big, C)) != SD_OK) return r;
     if ((r = run_linear(c, ctx, ctx_len, w.ctx_dim, W(pw, b.kv2), 2 * C, nullptr, nullptr, 0, s.kv, 2 * C)) != SD_OK)
       return r;
-    CK(sdk::launch_attention(s.big, C, s.kv, 2 * C, s.kv + C, 2 * C, s.ao, C, HW, ctx_len, heads, c.st));
+    CK(run_attn(c, s.big, C, s.kv, 2 * C, s.kv + C, 2 * C, s.ao, C, HW, ctx_len, heads));
     if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o2w), C, W(pw, b.o2b), s.t, C, s.t, C)) != SD_OK) return r;
     // GEGLU feed-forward: t += W2 (a * GELU(g)) + b2
-    CK(sdk::launch_layernorm(s.t, HW, C, W(pw, b.ln3g), W(pw, b.ln3b), ln_eps, s.nrm, c.st));
+    CK(run_ln(c, s.t, HW, C, W(pw, b.ln3g), W(pw, b.ln3b), ln_eps, s.nrm));
     if ((r = run_linear(c, s.nrm, HW, C, W(pw, b.f1w), 8 * C, W(pw, b.f1b), nullptr, 0, s.big, 4 * C,
                         sdk::GEMM_GEGLU)) != SD_OK)
       return r;
@@ -296,7 +342,10 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
 sd_status run_downsample(const Ctx& c, const ConvW& w, const void* pw, int H, int Wd, int C, const bf16* x, bf16* y,
                          bf16* planes) {
   const int Ho = H / 2, Wo = Wd / 2;
-  CK(sdk::launch_phase_split(x, H, Wd, C, planes, c.st));
+  {
+    sdp::Scope sc("phase_split", sdp::F_OTHER, 0, 4.0 * H * Wd * C, c.st);
+    CK(sdk::launch_phase_split(x, H, Wd, C, planes, c.st));
+  }
   GemmProblem p = base_problem(c);
   p.Ho = Ho;
   p.Wo = Wo;
@@ -320,20 +369,27 @@ sd_status run_downsample(const Ctx& c, const ConvW& w, const void* pw, int H, in
   p.epi.bias = W(pw, w.b);
   p.epi.out = y;
   p.epi.ld_out = C;
-  CK(sdk::gemm_tc_launch(p, c.st));
+  CK(launch_gemm(c, p));
   return SD_OK;
 }
 
 sd_status run_upsample(const Ctx& c, const ConvW& w, const void* pw, int H, int Wd, int C, const bf16* x, bf16* y,
                        bf16* up) {
-  CK(sdk::launch_upsample2x(x, H, Wd, C, up, c.st));
+  {
+    sdp::Scope sc("upsample2x", sdp::F_OTHER, 0, 10.0 * H * Wd * C, c.st);
+    CK(sdk::launch_upsample2x(x, H, Wd, C, up, c.st));
+  }
   return run_conv3x3(c, up, 2 * H, 2 * Wd, C, W(pw, w.w), C, W(pw, w.b), y);
 }
 
 sd_status run_conv_in(const Ctx& c, const ConvW& w, const void* pw, int kp, int H, int Wd, const bf16* s0, int c0,
                       const bf16* s1, int c1, const bf16* s2, int c2, int cout, bf16* y, bf16* col) {
-  CK(sdk::launch_conv_in_im2col(s0, c0, s1, c1, s2, c2, H, Wd, kp, col, c.st));
-  return run_linear(c, col, H * Wd, kp, W(pw, w.w), cout, W(pw, w.b), nullptr, 0, y, cout);
+  {
+    sdp::Scope sc("conv_in_im2col", sdp::F_OTHER, 0, 2.0 * H * Wd * (c0 + c1 + c2 + kp), c.st);
+    CK(sdk::launch_conv_in_im2col(s0, c0, s1, c1, s2, c2, H, Wd, kp, col, c.st));
+  }
+  return run_linear(c, col, H * Wd, kp, W(pw, w.w), cout, W(pw, w.b), nullptr, 0, y, cout, sdk::GEMM_PLAIN,
+                    9.0 * (c0 + c1 + c2));
 }
 
 sd_status run_output(const Ctx& c, const OutW& w, const void* pw, int H, int Wd, int C, int cout, int G, float eps,
@@ -345,7 +401,10 @@ sd_status run_output(const Ctx& c, const OutW& w, const void* pw, int H, int Wd,
 
 sd_status run_time(const Ctx& c, const TimeW& w, const void* pw, int proj, int temb_dim, float t, float* phi,
                    float* hid, float* temb) {
-  CK(sdk::launch_sinusoid(t, proj, phi, c.st));
+  {
+    sdp::Scope sc("sinusoid", sdp::F_OTHER, 0, 4.0 * proj, c.st);
+    CK(sdk::launch_sinusoid(t, proj, phi, c.st));
+  }
   sdk::GemvBatch b;
   memset(&b, 0, sizeof(b));
   b.njobs = 1;
@@ -353,12 +412,12 @@ sd_status run_time(const Ctx& c, const TimeW& w, const void* pw, int proj, int t
   b.silu_out = 1;
   b.x = phi;
   b.job[0] = {W(pw, w.l1w), W(pw, w.l1b), hid, temb_dim};
-  CK(sdk::launch_gemv(b, c.st));
+  CK(run_gemv(c, b));
   b.K = temb_dim;
   b.silu_out = 0;
   b.x = hid;
   b.job[0] = {W(pw, w.l2w), W(pw, w.l2b), temb, temb_dim};
-  CK(sdk::launch_gemv(b, c.st));
+  CK(run_gemv(c, b));
   return SD_OK;
 }
 
@@ -855,7 +914,7 @@ sd_status sd_resblock_fwd(const sd_resblock_cfg* cfg, const void* pw, const void
   b.silu_in = 1;
   b.x = temb;
   b.job[0] = {W(pw, w.tw), W(pw, w.tb), p.tproj, cfg->c_out};
-  CK(sdk::launch_gemv(b, p.c.st));
+  CK(run_gemv(p.c, b));
   return run_resblock(p.c, w, pw, cfg->height, cfg->width, static_cast<const bf16*>(x), cfg->c_x,
                       static_cast<const bf16*>(skip), cfg->c_skip, p.tproj, cfg->groups, cfg->eps,
                       static_cast<bf16*>(y), p.s);
@@ -929,7 +988,7 @@ sd_status sd_unet_step(const sd_unet_cfg* cfg, const void* pw, const void* laten
       b.x = p.temb;
       for (size_t i = i0; i < all_res.size() && b.njobs < sdk::kMaxGemvJobs; ++i)
         b.job[b.njobs++] = {W(pw, all_res[i]->tw), W(pw, all_res[i]->tb), tproj[i], all_res[i]->c_out};
-      CK(sdk::launch_gemv(b, c.st));
+      CK(run_gemv(c, b));
     }
   }
   size_t ri = 0;
