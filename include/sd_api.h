@@ -201,6 +201,26 @@ size_t sd_unet_workspace_size(const sd_unet_cfg* cfg);
 sd_status sd_time_embed(const sd_time_cfg* cfg, const void* packed_w, float timestep, float* temb_out,
                         void* workspace, size_t ws_bytes, sd_stream_t stream);
 
+/* Allocation-free variant of sd_time_embed. The source pages have no
+ * counterpart: it exists for callers that cannot give this library a workspace
+ * because they may not allocate device memory themselves, e.g. the enqueue step
+ * of a plugin inside another inference engine (the host engine owns every
+ * allocation) or a latency-critical loop where cudaMalloc/cudaFree would
+ * synchronise the device.
+ * Same arguments and result as sd_time_embed without the workspace: the two
+ * intermediate vectors live in a fixed device array of this library
+ * (2 x 4096 FP32 = 32 KiB, resident on every GPU that loads the library until
+ * the process exits). proj_dim and temb_dim above 4096 are rejected with
+ * SD_ERR_UNSUPPORTED before anything is launched. No device or host memory is
+ * allocated. The first call on a device looks up that array's device address
+ * (with the device current), so make the first call on each device before any
+ * stream capture. All calls share the one array: calls whose work overlaps on
+ * the GPU (different streams, or different host threads, without ordering)
+ * race on it; serialise them. Each call rewrites both vectors before reading
+ * them, so no state carries over between calls. */
+sd_status sd_time_embed_noalloc(const sd_time_cfg* cfg, const void* packed_w, float timestep, float* temb_out,
+                                sd_stream_t stream);
+
 /* SD_CONV_IN: x0 = latent [H, W, c_in] BF16, or for c_in = 9 the inpaint input
  *   assembled from x0 = noisy [H, W, 4], x1 = masked latent [H, W, 4],
  *   x2 = mask [H, W, 1] (channels in that order) without materialising it.

@@ -96,6 +96,7 @@ _SIGS = {
     "sd_transformer_workspace_size": (c_size_t, [POINTER(sd_transformer_cfg)]),
     "sd_unet_workspace_size": (c_size_t, [POINTER(sd_unet_cfg)]),
     "sd_time_embed": (c_int32, [POINTER(sd_time_cfg), _P, c_float, _P, _P, c_size_t, _P]),
+    "sd_time_embed_noalloc": (c_int32, [POINTER(sd_time_cfg), _P, c_float, _P, _P]),
     "sd_conv_fwd": (c_int32, [POINTER(sd_conv_cfg), c_int32, _P, _P, _P, _P, _P, _P, c_size_t, _P]),
     "sd_resblock_fwd": (c_int32, [POINTER(sd_resblock_cfg), _P, _P, _P, _P, _P, _P, c_size_t, _P]),
     "sd_transformer_fwd": (c_int32, [POINTER(sd_transformer_cfg), _P, _P, _P, _P, _P, c_size_t, _P]),
@@ -255,6 +256,13 @@ def sd_time_embed(cfg, packed_w, timestep, temb_out, workspace, ws_bytes, stream
     s = lib().sd_time_embed(ctypes.byref(cfg), _ptr(packed_w), float(timestep), _ptr(temb_out), _ptr(workspace),
                             int(ws_bytes), _stream(stream))
     return _check(s, "sd_time_embed") if check else s
+
+
+def sd_time_embed_noalloc(cfg, packed_w, timestep, temb_out, stream=None, check=True):
+    """Workspace-free time embedding (fixed device scratch inside the library)."""
+    s = lib().sd_time_embed_noalloc(ctypes.byref(cfg), _ptr(packed_w), float(timestep), _ptr(temb_out),
+                                    _stream(stream))
+    return _check(s, "sd_time_embed_noalloc") if check else s
 
 
 def sd_conv_fwd(cfg, kind, packed_w, x0, x1, x2, y, workspace, ws_bytes, stream=None, check=True):
