@@ -271,9 +271,10 @@ sd_status sd_query_device_status(void* workspace, sd_stream_t stream);
 typedef struct {
   char kernel[24];  /* "gemm_tc", "attention", "gn_stats", "gn_apply", "layernorm", "gemv", ... */
   int32_t family;   /* SD_FAMILY_* */
+  int32_t kernels;  /* kernels enqueued by this launch (a split-K GEMM enqueues 2) */
   double flops;
   double bytes;
-  float ms;
+  float ms;         /* device time between the two events */
 } sd_launch_record;
 
 enum {
@@ -282,7 +283,7 @@ enum {
 };
 
 sd_status sd_profile_begin(void);
-sd_status sd_profile_end(int32_t* n_launches);
+sd_status sd_profile_end(int32_t* n_kernels); /* kernels enqueued while recording */
 sd_status sd_profile_read(sd_launch_record* out, int32_t capacity, int32_t* n);
 
 /* Kernel launches issued by this library in this process so far. */

@@ -64,7 +64,7 @@ class sd_unet_cfg(ctypes.Structure):
 
 
 class sd_launch_record(ctypes.Structure):
-    _fields_ = [("kernel", c_char * 24), ("family", c_int32), ("flops", ctypes.c_double),
+    _fields_ = [("kernel", c_char * 24), ("family", c_int32), ("kernels", c_int32), ("flops", ctypes.c_double),
                 ("bytes", ctypes.c_double), ("ms", c_float)]
 
 
@@ -309,8 +309,8 @@ def sd_profile_read():
     _check(lib().sd_profile_read(None, 0, ctypes.byref(n)), "sd_profile_read")
     arr = (sd_launch_record * max(n.value, 1))()
     _check(lib().sd_profile_read(arr, n.value, ctypes.byref(n)), "sd_profile_read")
-    return [{"kernel": r.kernel.decode(), "family": FAMILY_NAMES.get(r.family, r.family), "flops": r.flops,
-             "bytes": r.bytes, "ms": r.ms} for r in arr[:n.value]]
+    return [{"kernel": r.kernel.decode(), "family": FAMILY_NAMES.get(r.family, r.family), "kernels": r.kernels,
+             "flops": r.flops, "bytes": r.bytes, "ms": r.ms} for r in arr[:n.value]]
 
 
 def sd_launch_count():

@@ -52,7 +52,7 @@ sd_status device_info(DevInfo* out) {
 // ------------------------------------------------------------------ workspace arena
 constexpr size_t kHeaderBytes = 256;
 constexpr int kMaxGroups = 64;
-constexpr int kMaxStatBlocks = 256;
+constexpr int kMaxStatBlocks = 512;  // GroupNorm partial-sum slots: 2 CTAs per SM, up to 256 SMs
 
 struct Arena {
   uint8_t* base;
@@ -73,8 +73,12 @@ struct Ctx {
   unsigned int* counter;
   float2* partial;
   float2* stats;
+  float* skws;  // split-K FP32 partial products
+  size_t skws_bytes;
   int sms;
 };
+
+constexpr size_t kSplitKBytes = size_t(16) << 20;
 
 // Header + GroupNorm scratch at the start of every workspace.
 Ctx make_ctx(Arena& ar, cudaStream_t st, int sms) {
@@ -84,8 +88,10 @@ Ctx make_ctx(Arena& ar, cudaStream_t st, int sms) {
   c.counter = h ? reinterpret_cast<unsigned int*>(h + 4) : nullptr;
   c.partial = static_cast<float2*>(ar.take(sizeof(float2) * kMaxGroups * kMaxStatBlocks));
   c.stats = static_cast<float2*>(ar.take(sizeof(float2) * kMaxGroups));
+  c.skws = static_cast<float*>(ar.take(kSplitKBytes));
+  c.skws_bytes = kSplitKBytes;
   c.st = st;
-  c.sms = sms < kMaxStatBlocks ? sms : kMaxStatBlocks;
+  c.sms = sms < kMaxStatBlocks / 2 ? sms : kMaxStatBlocks / 2;
   return c;
 }
 
@@ -139,7 +145,7 @@ int launch_gemm(const Ctx& c, const GemmProblem& p, double alg_k = 0) {
   for (int i = 0; i < p.nb; ++i) by += 2.0 * p.b[i].K * (p.b[i].rows < p.N ? p.b[i].rows : p.N);
   by += 2.0 * M * (p.epi.mode == sdk::GEMM_GEGLU ? p.N / 2 : p.N);
   if (p.epi.residual) by += 2.0 * M * p.N;
-  sdp::Scope sc("gemm_tc", sdp::F_GEMM, fl, by, c.st);
+  sdp::Scope sc("gemm_tc", sdp::F_GEMM, fl, by, c.st, sdk::gemm_tc_plan_launches(p));
   return sdk::gemm_tc_launch(p, c.st);
 }
 
@@ -147,6 +153,8 @@ GemmProblem base_problem(const Ctx& c) {
   GemmProblem p;
   memset(&p, 0, sizeof(p));
   p.err = c.err;
+  p.splitk_ws = c.skws;
+  p.splitk_ws_bytes = c.skws_bytes;
   return p;
 }
 
@@ -299,11 +307,14 @@ int run_ln(const Ctx& c, const bf16* x, int N, int C, const bf16* g, const bf16*
   return sdk::launch_layernorm(x, N, C, g, b, eps, y, c.st);
 }
 
-int run_attn(const Ctx& c, const bf16* q, int ldq, const bf16* k, int ldk, const bf16* v, int ldv, bf16* o, int ldo,
-             int Nq, int Nk, int heads) {
+// Attention of Q (rows of qbase, columns q_col + 64h) against K/V (rows of
+// kvbase, columns k_col + 64h and v_col + 64h), head_dim 64, into O [Nq, ldo].
+int run_attn(const Ctx& c, const bf16* qbase, int q_ld, int q_col, const bf16* kvbase, int kv_ld, int k_col,
+             int v_col, bf16* o, int ldo, int Nq, int Nk, int heads) {
   const double C = 64.0 * heads;
   sdp::Scope sc("attention", sdp::F_ATTN, 4.0 * Nq * Nk * C, 2.0 * C * (2.0 * Nq + 2.0 * Nk), c.st);
-  return sdk::launch_attention(q, ldq, k, ldk, v, ldv, o, ldo, Nq, Nk, heads, c.st);
+  return sdk::launch_attention_tc(qbase, q_ld, Nq, q_col, kvbase, kv_ld, Nk, k_col, v_col, o, ldo, Nq, Nk, heads,
+                                  c.err, c.st);
 }
 
 // Transformer2DModel; y may alias x.
@@ -319,14 +330,14 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
     // self-attention: t += Wo Attn(LN1(t))
     CK(run_ln(c, s.t, HW, C, W(pw, b.ln1g), W(pw, b.ln1b), ln_eps, s.nrm));
     if ((r = run_linear(c, s.nrm, HW, C, W(pw, b.qkv), 3 * C, nullptr, nullptr, 0, s.big, 3 * C)) != SD_OK) return r;
-    CK(run_attn(c, s.big, 3 * C, s.big + C, 3 * C, s.big + 2 * C, 3 * C, s.ao, C, HW, HW, heads));
+    CK(run_attn(c, s.big, 3 * C, 0, s.big, 3 * C, C, 2 * C, s.ao, C, HW, HW, heads));
     if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o1w), C, W(pw, b.o1b), s.t, C, s.t, C)) != SD_OK) return r;
     // cross-attention: t += Wo' Attn(LN2(t), ctx)
     CK(run_ln(c, s.t, HW, C, W(pw, b.ln2g), W(pw, b.ln2b), ln_eps, s.nrm));
     if ((r = run_linear(c, s.nrm, HW, C, W(pw, b.q2), C, nullptr, nullptr, 0, s.big, C)) != SD_OK) return r;
     if ((r = run_linear(c, ctx, ctx_len, w.ctx_dim, W(pw, b.kv2), 2 * C, nullptr, nullptr, 0, s.kv, 2 * C)) != SD_OK)
       return r;
-    CK(run_attn(c, s.big, C, s.kv, 2 * C, s.kv + C, 2 * C, s.ao, C, HW, ctx_len, heads));
+    CK(run_attn(c, s.big, C, 0, s.kv, 2 * C, 0, C, s.ao, C, HW, ctx_len, heads));
     if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o2w), C, W(pw, b.o2b), s.t, C, s.t, C)) != SD_OK) return r;
     // GEGLU feed-forward: t += W2 (a * GELU(g)) + b2
     CK(run_ln(c, s.t, HW, C, W(pw, b.ln3g), W(pw, b.ln3b), ln_eps, s.nrm));

@@ -7,7 +7,34 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace sdk {
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel is launched with programmatic stream serialisation: it may start
+// while the previous kernel on the stream finishes, runs its prologue (barrier
+// init, TMEM allocation, descriptor prefetch), and waits in pdl_wait() before
+// its first global-memory access, reads or writes. pdl_trigger() lets the next
+// kernel start launching once every CTA of this one has started.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Workspace header: word 0 = device error flags (bit set per failing kernel family).
 enum : int { ERR_MBAR_TIMEOUT = 1, ERR_BAD_ARGS = 2 };

@@ -28,8 +28,10 @@ struct __align__(64) GemmMaps {
 struct GemmArgs {
   int32_t Ho, Wo, BH, BW, tiles_x, N;
   int32_t nseg, total_kb;
+  int32_t kb_per_split;  // k-blocks per blockIdx.z (== total_kb without split-K)
   GemmSeg seg[kGemmMaxSeg];
   GemmEpi epi;
+  float* partial;  // split-K: FP32 [gridDim.z][Ho*Wo][N]; null otherwise
   int* err;
 };
 
@@ -79,17 +81,25 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // everything above touched only shared memory and TMEM: wait for the previous kernel here
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
       for (int i = 0; i < kGemmMaxA; ++i) tma_prefetch_desc(&maps.a[i]);
       tma_prefetch_desc(&maps.b[0]);
       tma_prefetch_desc(&maps.b[1]);
-      int kb = 0;
+      const int kb_lo = blockIdx.z * args.kb_per_split;
+      const int kb_hi = min(args.total_kb, kb_lo + args.kb_per_split);
+      int g = 0;  // position in the whole reduction
       bool ok = true;
-      for (int si = 0; si < args.nseg && ok; ++si) {
+      for (int si = 0; si < args.nseg && ok && g < kb_hi; ++si) {
         const GemmSeg sg = args.seg[si];
-        for (int j = 0; j < sg.nkb; ++j, ++kb) {
+        for (int j = 0; j < sg.nkb; ++j, ++g) {
+          if (g < kb_lo) continue;
+          if (g >= kb_hi) break;
+          const int kb = g - kb_lo;
           const int s = kb % STAGES;
           const int it = kb / STAGES;
           if (kb >= STAGES && !mbar_wait(&empty_bar[s], (it - 1) & 1, abort_flag, args.err)) {
@@ -108,7 +118,9 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       bool ok = true;
-      for (int kb = 0; kb < args.total_kb; ++kb) {
+      const int kb_lo = blockIdx.z * args.kb_per_split;
+      const int nkb = min(args.total_kb, kb_lo + args.kb_per_split) - kb_lo;
+      for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % STAGES;
         const int it = kb / STAGES;
         if (!mbar_wait(&full_bar[s], it & 1, abort_flag, args.err)) {
@@ -135,7 +147,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int c = et; c < BN; c += 128) {
       const int n = n0 + c;
       float v = 0.f;
-      if (n < args.N) {
+      if (n < args.N && !args.partial) {
         if (args.epi.bias) v += __bfloat162float(args.epi.bias[n]);
         if (args.epi.bias2) v += __bfloat162float(args.epi.bias2[n]);
         if (args.epi.colvec) v += args.epi.colvec[n];
@@ -163,6 +175,19 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + epi_col[cc * 32 + j];
       const bool full = (nb + 32 <= args.N);
+      if (args.partial) {
+        float* dst = args.partial + ((size_t)blockIdx.z * args.Ho * args.Wo + grow) * args.N + nb;
+        if (full) {
+          float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) d4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (nb + j < args.N) dst[j] = v[j];
+        }
+        continue;
+      }
       if (args.epi.mode == GEMM_GEGLU) {
         // columns (2j, 2j+1) hold (value_j, gate_j); output column (nb/2 + j)
         uint32_t o[8];
@@ -232,6 +257,50 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
+// Split-K reduction: out = epilogue(sum over splits of partial), 8 columns per
+// thread, splits added in index order (deterministic).
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N, GemmEpi epi) {
+  pdl_wait();
+  pdl_trigger();
+  const int V = N / 8;
+  const size_t total = (size_t)M * V;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int row = (int)(i / V);
+    const int c = (int)(i % V) * 8;
+    float v[8];
+    const float4* p0 = reinterpret_cast<const float4*>(partial + (size_t)row * N + c);
+    float4 a = p0[0], b = p0[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    for (int z = 1; z < splits; ++z) {
+      const float4* pz = reinterpret_cast<const float4*>(partial + ((size_t)z * M + row) * N + c);
+      a = pz[0];
+      b = pz[1];
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w; v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float add = 0.f;
+      if (epi.bias) add += __bfloat162float(epi.bias[c + j]);
+      if (epi.bias2) add += __bfloat162float(epi.bias2[c + j]);
+      if (epi.colvec) add += epi.colvec[c + j];
+      v[j] += add;
+    }
+    if (epi.mode == GEMM_GEGLU) {
+      const uint32_t o0 = pack_bf16x2(v[0] * gelu_erf(v[1]), v[2] * gelu_erf(v[3]));
+      const uint32_t o1 = pack_bf16x2(v[4] * gelu_erf(v[5]), v[6] * gelu_erf(v[7]));
+      *reinterpret_cast<uint2*>(epi.out + (size_t)row * epi.ld_out + c / 2) = make_uint2(o0, o1);
+      continue;
+    }
+    if (epi.residual) {
+      const uint4 r = *reinterpret_cast<const uint4*>(epi.residual + (size_t)row * epi.ld_res + c);
+      v[0] += bf16lo(r.x); v[1] += bf16hi(r.x); v[2] += bf16lo(r.y); v[3] += bf16hi(r.y);
+      v[4] += bf16lo(r.z); v[5] += bf16hi(r.z); v[6] += bf16lo(r.w); v[7] += bf16hi(r.w);
+    }
+    *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
+}
+
 // ------------------------------------------------------------------ host side
 
 namespace {
@@ -281,7 +350,8 @@ bool tmap_encode_4d(CUtensorMap* m, const void* ptr, const uint64_t d[4], uint32
 }
 
 template <int BN, int STAGES>
-static int launch_bn(const GemmMaps& maps, const GemmArgs& args, int tiles_m, int tiles_n, cudaStream_t st) {
+static int launch_bn(const GemmMaps& maps, const GemmArgs& args, int tiles_m, int tiles_n, int splits,
+                     cudaStream_t st) {
   constexpr int kStageBytes = kATileBytes + BN * kBK * 2;
   constexpr size_t smem = 1024 + (size_t)STAGES * kStageBytes + 256 + BN * 4;
   static bool attr_set = false;  // benign race: the attribute value is identical for every caller
@@ -291,8 +361,7 @@ static int launch_bn(const GemmMaps& maps, const GemmArgs& args, int tiles_m, in
     if (e != cudaSuccess) return (int)e;
     attr_set = true;
   }
-  gemm_tc_kernel<BN, STAGES><<<dim3(tiles_m, tiles_n), 192, smem, st>>>(maps, args);
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(gemm_tc_kernel<BN, STAGES>, dim3(tiles_m, tiles_n, splits), dim3(192), smem, st, maps, args);
 }
 
 static void choose_tile_rect(int Ho, int Wo, int* BH, int* BW) {
@@ -326,7 +395,11 @@ static int choose_bn(int N, int tiles_m, int num_sms) {
   return 0;
 }
 
-int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
+struct GemmPlan {
+  int BH, BW, tiles_x, tiles_m, bn, tiles_n, splits, kb_per_split, total_kb;
+};
+
+static int sm_count() {
   static int num_sms = 0;
   if (num_sms == 0) {
     int dev = 0;
@@ -334,28 +407,72 @@ int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
     cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (num_sms <= 0) num_sms = 148;
   }
+  return num_sms;
+}
+
+// Tile shape, N tile and split-K factor for a problem.
+static bool plan_gemm(const GemmProblem& p, GemmPlan* g) {
+  const int sms = sm_count();
+  choose_tile_rect(p.Ho, p.Wo, &g->BH, &g->BW);
+  g->tiles_x = (p.Wo + g->BW - 1) / g->BW;
+  g->tiles_m = g->tiles_x * ((p.Ho + g->BH - 1) / g->BH);
+  g->total_kb = 0;
+  for (int i = 0; i < p.nseg; ++i) g->total_kb += p.seg[i].nkb;
+  g->bn = p.force_bn ? p.force_bn : choose_bn(p.N, g->tiles_m, sms);
+  if (g->bn == 0 || g->total_kb <= 0) return false;
+  g->splits = 1;
+  // under-filled grid with a long reduction: a 128-wide N tile and split-K
+  const bool small = (long)g->tiles_m * (p.N / 64 > 0 ? p.N / 64 : 1) < sms && g->total_kb >= 16 && p.N % 128 == 0;
+  if (p.force_splits > 0) {
+    g->splits = p.force_splits;
+  } else if (small && p.splitk_ws && !p.force_bn) {
+    g->bn = 128;
+    const int ctas = g->tiles_m * (p.N / 128);
+    int sp = (sms + ctas - 1) / ctas;
+    if (sp > g->total_kb / 4) sp = g->total_kb / 4;
+    if (sp > 16) sp = 16;
+    const size_t per = (size_t)p.Ho * p.Wo * p.N * sizeof(float);
+    while (sp > 1 && per * sp > p.splitk_ws_bytes) --sp;
+    g->splits = sp < 1 ? 1 : sp;
+  }
+  g->tiles_n = (p.N + g->bn - 1) / g->bn;
+  g->kb_per_split = (g->total_kb + g->splits - 1) / g->splits;
+  g->splits = (g->total_kb + g->kb_per_split - 1) / g->kb_per_split;  // no empty split
+  if (g->splits > 1 && (!p.splitk_ws || (size_t)p.Ho * p.Wo * p.N * sizeof(float) * g->splits > p.splitk_ws_bytes ||
+                        p.N % 8))
+    return false;
+  return true;
+}
+
+int gemm_tc_plan_launches(const GemmProblem& p) {
+  GemmPlan g;
+  if (!plan_gemm(p, &g)) return 1;
+  return g.splits > 1 ? 2 : 1;
+}
+
+int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
+  if (p.nseg <= 0 || p.nseg > kGemmMaxSeg || p.na <= 0 || p.na > kGemmMaxA || p.nb <= 0 || p.nb > kGemmMaxB)
+    return -1;
+  GemmPlan g;
+  if (!plan_gemm(p, &g)) return -1;
   GemmArgs args{};
   args.Ho = p.Ho;
   args.Wo = p.Wo;
-  choose_tile_rect(p.Ho, p.Wo, &args.BH, &args.BW);
-  args.tiles_x = (p.Wo + args.BW - 1) / args.BW;
-  const int tiles_y = (p.Ho + args.BH - 1) / args.BH;
-  const int tiles_m = args.tiles_x * tiles_y;
+  args.BH = g.BH;
+  args.BW = g.BW;
+  args.tiles_x = g.tiles_x;
   args.N = p.N;
   args.nseg = p.nseg;
-  args.total_kb = 0;
-  if (p.nseg <= 0 || p.nseg > kGemmMaxSeg || p.na <= 0 || p.na > kGemmMaxA || p.nb <= 0 || p.nb > kGemmMaxB)
-    return -1;
-  for (int i = 0; i < p.nseg; ++i) {
-    args.seg[i] = p.seg[i];
-    args.total_kb += p.seg[i].nkb;
-  }
-  if (args.total_kb <= 0) return -1;
+  for (int i = 0; i < p.nseg; ++i) args.seg[i] = p.seg[i];
+  args.total_kb = g.total_kb;
+  args.kb_per_split = g.kb_per_split;
   args.epi = p.epi;
+  args.partial = g.splits > 1 ? p.splitk_ws : nullptr;
   args.err = p.err;
-  const int bn = p.force_bn ? p.force_bn : choose_bn(p.N, tiles_m, num_sms);
-  if (bn == 0) return -1;
-  const int tiles_n = (p.N + bn - 1) / bn;
+  const int bn = g.bn;
+  const int tiles_m = g.tiles_m;
+  const int tiles_n = g.tiles_n;
+  const int splits = g.splits;
 
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
@@ -368,15 +485,23 @@ int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
     const GemmBSrc& b = p.b[i < p.nb ? i : 0];
     if (!tmap_encode_2d(&maps.b[i], b.ptr, (uint64_t)b.K, (uint64_t)b.rows, 64, (uint32_t)bn)) return -2;
   }
+  int e;
   switch (bn) {
-    case 32: return launch_bn<32, 6>(maps, args, tiles_m, tiles_n, stream);
-    case 64: return launch_bn<64, 4>(maps, args, tiles_m, tiles_n, stream);
-    case 128: return launch_bn<128, 3>(maps, args, tiles_m, tiles_n, stream);
-    case 160: return launch_bn<160, 3>(maps, args, tiles_m, tiles_n, stream);
-    case 192: return launch_bn<192, 4>(maps, args, tiles_m, tiles_n, stream);
-    case 256: return launch_bn<256, 4>(maps, args, tiles_m, tiles_n, stream);
+    case 32: e = launch_bn<32, 6>(maps, args, tiles_m, tiles_n, splits, stream); break;
+    case 64: e = launch_bn<64, 4>(maps, args, tiles_m, tiles_n, splits, stream); break;
+    case 128: e = launch_bn<128, 3>(maps, args, tiles_m, tiles_n, splits, stream); break;
+    case 160: e = launch_bn<160, 3>(maps, args, tiles_m, tiles_n, splits, stream); break;
+    case 192: e = launch_bn<192, 4>(maps, args, tiles_m, tiles_n, splits, stream); break;
+    case 256: e = launch_bn<256, 4>(maps, args, tiles_m, tiles_n, splits, stream); break;
     default: return -1;
   }
+  if (e != 0 || splits <= 1) return e;
+  const int M = p.Ho * p.Wo;
+  const size_t vecs = (size_t)M * (p.N / 8);
+  int blocks = (int)((vecs + 255) / 256);
+  if (blocks > sm_count() * 8) blocks = sm_count() * 8;
+  return (int)launch_pdl(splitk_reduce_kernel, dim3(blocks), dim3(256), 0, stream, (const float*)p.splitk_ws, splits, M,
+                         p.N, p.epi);
 }
 
 }  // namespace sdk

@@ -50,6 +50,9 @@ struct GemmEpi {
 };
 
 // A full problem: output grid Ho x Wo (M = Ho*Wo rows), N output features.
+// When the tile grid cannot fill the GPU and an FP32 split-K buffer is given,
+// the reduction is split over blockIdx.z and a second kernel adds the partial
+// products in a fixed order and applies the epilogue.
 struct GemmProblem {
   int32_t Ho, Wo, N;
   int32_t na, nb, nseg;
@@ -58,8 +61,14 @@ struct GemmProblem {
   GemmSeg seg[kGemmMaxSeg];
   GemmEpi epi;
   int* err;
-  int32_t force_bn;  // 0 = heuristic
+  int32_t force_bn;      // 0 = heuristic
+  int32_t force_splits;  // 0 = heuristic, 1 = no split
+  float* splitk_ws;      // FP32 partials [splits][Ho*Wo][N], or null
+  size_t splitk_ws_bytes;
 };
+
+// Number of kernels gemm_tc_launch will enqueue for p (1, or 2 with split-K).
+int gemm_tc_plan_launches(const GemmProblem& p);
 
 // Launch on `stream`. Returns 0 on success, a cudaError_t value otherwise
 // (or -1 for an unsupported shape).

@@ -51,7 +51,14 @@ int launch_conv_in_im2col(const __nv_bfloat16* s0, int c0, const __nv_bfloat16* 
                           const __nv_bfloat16* s2, int c2, int H, int W, int Kp, __nv_bfloat16* y,
                           cudaStream_t st);
 
-// Flash attention (head_dim 64): O[i, h*64 + d] = softmax_j(Q_i.K_j / 8) V_j per head.
+// Flash attention on tcgen05 (head_dim 64): O[i, h*64 + d] = softmax_j(Q_i.K_j / 8) V_j
+// per head; Q rows come from a [q_rows, q_ld] matrix at column q_col + 64h, K and V
+// from a [kv_rows, kv_ld] matrix at columns k_col + 64h and v_col + 64h.
+int launch_attention_tc(const __nv_bfloat16* qbase, int q_ld, int q_rows, int q_col, const __nv_bfloat16* kvbase,
+                        int kv_ld, int kv_rows, int k_col, int v_col, __nv_bfloat16* O, int ldo, int Nq, int Nk,
+                        int heads, int* err, cudaStream_t st);
+
+// Flash attention (head_dim 64) on mma.sync: O[i, h*64 + d] = softmax_j(Q_i.K_j / 8) V_j per head.
 int launch_attention(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk, const __nv_bfloat16* V,
                      int ldv, __nv_bfloat16* O, int ldo, int Nq, int Nk, int heads, cudaStream_t st);
 

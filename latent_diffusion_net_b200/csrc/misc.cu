@@ -9,6 +9,8 @@ namespace sdk {
 // Sinusoidal time embedding (tutorial page, sinusoidal embedding paragraph):
 // [cos(t f_i) | sin(t f_i)], f_i = exp(-ln(10000) i / half), evaluated in FP64.
 __global__ void sinusoid_kernel(float t, int half, float* out) {
+  pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= half) return;
   const double f = exp(-9.210340371976184 * (double)i / (double)half);  // ln(10000)
@@ -19,14 +21,15 @@ __global__ void sinusoid_kernel(float t, int half, float* out) {
 
 int launch_sinusoid(float t, int proj_dim, float* out, cudaStream_t st) {
   const int half = proj_dim / 2;
-  sinusoid_kernel<<<(half + 127) / 128, 128, 0, st>>>(t, half, out);
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(sinusoid_kernel, dim3((half + 127) / 128), dim3(128), 0, st, t, half, out);
 }
 
 // Grouped GEMV: one warp per output row, 16-byte weight loads, x staged in
 // shared memory with the optional input SiLU applied once.
 __global__ void gemv_kernel(const __grid_constant__ GemvBatch batch) {
   extern __shared__ float xs[];
+  pdl_wait();
+  pdl_trigger();
   for (int k = threadIdx.x; k < batch.K; k += blockDim.x) {
     const float v = batch.x[k];
     xs[k] = batch.silu_in ? silu_f(v) : v;
@@ -63,12 +66,13 @@ int launch_gemv(const GemvBatch& batch, cudaStream_t st) {
   const int warps = 8;
   const int blocks = (int)((rows + warps - 1) / warps);
   if (blocks == 0) return 0;
-  gemv_kernel<<<blocks, warps * 32, batch.K * sizeof(float), st>>>(batch);
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(gemv_kernel, dim3(blocks), dim3(warps * 32), batch.K * sizeof(float), st, batch);
 }
 
 // Nearest 2x (UpSample bullet): y[i][j] = x[i/2][j/2], one 16-byte vector per thread.
 __global__ void upsample2x_kernel(const uint4* __restrict__ x, int H, int W, int V, uint4* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const size_t total = (size_t)4 * H * W * V;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
        idx += (size_t)gridDim.x * blockDim.x) {
@@ -85,12 +89,14 @@ int launch_upsample2x(const __nv_bfloat16* x, int H, int W, int C, __nv_bfloat16
   const size_t total = (size_t)4 * H * W * V;
   int blocks = (int)((total + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
-  upsample2x_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), H, W, V, reinterpret_cast<uint4*>(y));
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(upsample2x_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4*>(x), H, W,
+                         V, reinterpret_cast<uint4*>(y));
 }
 
 // Phase split: plane (a, b) holds the pixels (2i + a, 2j + b).
 __global__ void phase_split_kernel(const uint4* __restrict__ x, int H, int W, int V, uint4* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int Ho = H / 2, Wo = W / 2;
   const size_t total = (size_t)H * W * V;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
@@ -109,14 +115,16 @@ int launch_phase_split(const __nv_bfloat16* x, int H, int W, int C, __nv_bfloat1
   const size_t total = (size_t)H * W * V;
   int blocks = (int)((total + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
-  phase_split_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(x), H, W, V, reinterpret_cast<uint4*>(y));
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(phase_split_kernel, dim3(blocks), dim3(256), 0, st, reinterpret_cast<const uint4*>(x), H, W,
+                         V, reinterpret_cast<uint4*>(y));
 }
 
 // conv_in operand (small C_in): one thread per output element.
 __global__ void conv_in_im2col_kernel(const __nv_bfloat16* __restrict__ s0, int c0, const __nv_bfloat16* __restrict__ s1,
                                       int c1, const __nv_bfloat16* __restrict__ s2, int c2, int H, int W, int Kp,
                                       __nv_bfloat16* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int Cin = c0 + c1 + c2;
   const size_t total = (size_t)H * W * Kp;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total;
@@ -149,8 +157,7 @@ int launch_conv_in_im2col(const __nv_bfloat16* s0, int c0, const __nv_bfloat16* 
   const size_t total = (size_t)H * W * Kp;
   int blocks = (int)((total + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
-  conv_in_im2col_kernel<<<blocks, 256, 0, st>>>(s0, c0, s1, c1, s2, c2, H, W, Kp, y);
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(conv_in_im2col_kernel, dim3(blocks), dim3(256), 0, st, s0, c0, s1, c1, s2, c2, H, W, Kp, y);
 }
 
 }  // namespace sdk

@@ -24,6 +24,8 @@ __global__ void gn_stats_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
                                 unsigned int* __restrict__ counter, float2* __restrict__ stats) {
   extern __shared__ float4 red[];  // [blockDim.x]
   __shared__ bool is_last;
+  pdl_wait();
+  pdl_trigger();
   const int C = C0 + C1;
   const int V = C >> 3;
   const int cpg = C / G;
@@ -47,8 +49,7 @@ __global__ void gn_stats_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
       base = x1 + (c - C0);
       ld = C1;
     }
-    for (int p = p0 + pi; p < p1; p += ppi) {
-      const uint4 w = *reinterpret_cast<const uint4*>(base + (size_t)p * ld);
+    auto acc = [&](const uint4 w) {
       const float f[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
                           bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
 #pragma unroll
@@ -61,7 +62,20 @@ __global__ void gn_stats_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
           qb += f[j] * f[j];
         }
       }
+    };
+    int p = p0 + pi;
+    // four independent 16-byte loads in flight per thread
+    for (; p + 3 * ppi < p1; p += 4 * ppi) {
+      const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(base + (size_t)p * ld));
+      const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(base + (size_t)(p + ppi) * ld));
+      const uint4 w2 = __ldg(reinterpret_cast<const uint4*>(base + (size_t)(p + 2 * ppi) * ld));
+      const uint4 w3 = __ldg(reinterpret_cast<const uint4*>(base + (size_t)(p + 3 * ppi) * ld));
+      acc(w0);
+      acc(w1);
+      acc(w2);
+      acc(w3);
     }
+    for (; p < p1; p += ppi) acc(__ldg(reinterpret_cast<const uint4*>(base + (size_t)p * ld)));
   }
   red[t] = make_float4(sa, qa, sb, qb);
   __syncthreads();
@@ -139,6 +153,8 @@ __global__ void gn_apply_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
                                 const __nv_bfloat16* __restrict__ gamma, const __nv_bfloat16* __restrict__ beta,
                                 int silu, __nv_bfloat16* __restrict__ y) {
   extern __shared__ float2 ab[];  // per channel (scale, shift)
+  pdl_wait();
+  pdl_trigger();
   const int C = C0 + C1;
   const int cpg = C / G;
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
@@ -175,6 +191,8 @@ constexpr int kLnMaxVecPerLane = 8;
 
 __global__ void ln_kernel(const __nv_bfloat16* __restrict__ x, int N, int C, const __nv_bfloat16* __restrict__ gamma,
                           const __nv_bfloat16* __restrict__ beta, float eps, __nv_bfloat16* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= N) return;
@@ -236,9 +254,10 @@ __global__ void ln_kernel(const __nv_bfloat16* __restrict__ x, int N, int C, con
 int gn_stats_blocks(int HW, int C, int num_sms) {
   const int V = C / 8;
   const int ppi = V >= 256 ? 1 : 256 / V;
-  int nblk = HW / (ppi * 4);
+  // about 8 pixels per thread, at most two CTAs per SM
+  int nblk = HW / (ppi * 8);
   if (nblk < 1) nblk = 1;
-  if (nblk > num_sms) nblk = num_sms;
+  if (nblk > 2 * num_sms) nblk = 2 * num_sms;
   return nblk;
 }
 
@@ -249,9 +268,8 @@ int launch_gn_stats(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, in
   const int ppi = V >= 256 ? 1 : 256 / V;
   const int threads = V * ppi;
   const int nblk = gn_stats_blocks(HW, C, num_sms);
-  gn_stats_kernel<<<nblk, threads, threads * sizeof(float4), st>>>(x0, C0, x1, C1, HW, G, ppi, eps, partial,
-                                                                  counter, stats);
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(gn_stats_kernel, dim3(nblk), dim3(threads), threads * sizeof(float4), st, x0, C0, x1, C1, HW,
+                         G, ppi, eps, partial, counter, stats);
 }
 
 int launch_gn_apply(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G,
@@ -261,16 +279,15 @@ int launch_gn_apply(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, in
   const size_t total = (size_t)HW * (C / 8);
   int blocks = (int)((total + 255) / 256);
   if (blocks > num_sms * 8) blocks = num_sms * 8;
-  gn_apply_kernel<<<blocks, 256, C * sizeof(float2), st>>>(x0, C0, x1, C1, HW, G, stats, gamma, beta, silu, y);
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(gn_apply_kernel, dim3(blocks), dim3(256), C * sizeof(float2), st, x0, C0, x1, C1, HW, G,
+                         stats, gamma, beta, silu, y);
 }
 
 int launch_layernorm(const __nv_bfloat16* x, int N, int C, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,
                      float eps, __nv_bfloat16* y, cudaStream_t st) {
   const int warps_per_block = 8;
   const int blocks = (N + warps_per_block - 1) / warps_per_block;
-  ln_kernel<<<blocks, warps_per_block * 32, 0, st>>>(x, N, C, gamma, beta, eps, y);
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(ln_kernel, dim3(blocks), dim3(warps_per_block * 32), 0, st, x, N, C, gamma, beta, eps, y);
 }
 
 }  // namespace sdk

@@ -16,12 +16,14 @@ std::atomic<long long> g_launches{0};
 struct Rec {
   char kernel[24];
   int family;
+  int kernels;
   double flops, bytes;
 };
 
 struct Recorder {
   bool on = false;
   size_t idx = 0;
+  long long kernels = 0;
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> ev;  // 2 per record, reused across recordings
 };
@@ -36,11 +38,12 @@ bool capturing(cudaStream_t st) {
 
 }  // namespace
 
-Scope::Scope(const char* kernel, int family, double flops, double bytes, cudaStream_t st)
+Scope::Scope(const char* kernel, int family, double flops, double bytes, cudaStream_t st, int kernels)
     : slot_(-1), flags_(0), st_(st) {
-  g_launches.fetch_add(1, std::memory_order_relaxed);
+  g_launches.fetch_add(kernels, std::memory_order_relaxed);
   Recorder& r = t_rec;
   if (!r.on) return;
+  r.kernels += kernels;
   const size_t i = r.idx;
   if (2 * i + 1 >= r.ev.size()) {
     if (capturing(st)) return;  // events are only created outside capture
@@ -55,6 +58,7 @@ Scope::Scope(const char* kernel, int family, double flops, double bytes, cudaStr
   memset(rc.kernel, 0, sizeof(rc.kernel));
   strncpy(rc.kernel, kernel, sizeof(rc.kernel) - 1);
   rc.family = family;
+  rc.kernels = kernels;
   rc.flops = flops;
   rc.bytes = bytes;
   // inside stream capture a plain event record only expresses a dependency;
@@ -77,12 +81,13 @@ extern "C" {
 sd_status sd_profile_begin(void) {
   sdp::t_rec.on = true;
   sdp::t_rec.idx = 0;
+  sdp::t_rec.kernels = 0;
   return SD_OK;
 }
 
-sd_status sd_profile_end(int32_t* n_launches) {
+sd_status sd_profile_end(int32_t* n_kernels) {
   sdp::t_rec.on = false;
-  if (n_launches) *n_launches = (int32_t)sdp::t_rec.idx;
+  if (n_kernels) *n_kernels = (int32_t)sdp::t_rec.kernels;
   return SD_OK;
 }
 
@@ -96,6 +101,7 @@ sd_status sd_profile_read(sd_launch_record* out, int32_t capacity, int32_t* n) {
     memset(&o, 0, sizeof(o));
     memcpy(o.kernel, r.recs[i].kernel, sizeof(o.kernel));
     o.family = r.recs[i].family;
+    o.kernels = r.recs[i].kernels;
     o.flops = r.recs[i].flops;
     o.bytes = r.recs[i].bytes;
     float ms = -1.f;

@@ -13,7 +13,8 @@ enum Family : int { F_GEMM = 0, F_ATTN = 1, F_GN_STATS = 2, F_GN_APPLY = 3, F_LN
 
 class Scope {
  public:
-  Scope(const char* kernel, int family, double flops, double bytes, cudaStream_t st);
+  // `kernels`: how many kernels the bracketed launch enqueues
+  Scope(const char* kernel, int family, double flops, double bytes, cudaStream_t st, int kernels = 1);
   ~Scope();
 
  private:
