@@ -50,8 +50,10 @@ sd_status device_info(DevInfo* out) {
 }
 
 // ------------------------------------------------------------------ workspace arena
-constexpr size_t kHeaderBytes = 256;
+constexpr size_t kHeaderBytes = 256;   // word 0: device error flags
+constexpr int kMaxGnLaunches = 256;      // GroupNorm statistics slots per call
 constexpr int kMaxGroups = 64;
+constexpr size_t kGnAccBytes = (size_t)kMaxGnLaunches * 2 * kMaxGroups * sizeof(unsigned long long);
 constexpr int kMaxStatBlocks = 512;  // GroupNorm partial-sum slots: 2 CTAs per SM, up to 256 SMs
 
 struct Arena {
@@ -70,9 +72,8 @@ struct Arena {
 struct Ctx {
   cudaStream_t st;
   int* err;
-  unsigned int* counter;
-  float2* partial;
-  float2* stats;
+  unsigned long long* gn_acc;  // [kMaxGnLaunches][2 * kMaxGroups], zeroed at the start of every call
+  int* gn_seq;                 // host: GroupNorm launches issued so far in this call
   float* skws;  // split-K FP32 partial products
   size_t skws_bytes;
   int sms;
@@ -83,11 +84,10 @@ constexpr size_t kSplitKBytes = size_t(16) << 20;
 // Header + GroupNorm scratch at the start of every workspace.
 Ctx make_ctx(Arena& ar, cudaStream_t st, int sms) {
   Ctx c;
-  uint8_t* h = static_cast<uint8_t*>(ar.take(kHeaderBytes));
+  uint8_t* h = static_cast<uint8_t*>(ar.take(kHeaderBytes + kGnAccBytes));
   c.err = reinterpret_cast<int*>(h);
-  c.counter = h ? reinterpret_cast<unsigned int*>(h + 4) : nullptr;
-  c.partial = static_cast<float2*>(ar.take(sizeof(float2) * kMaxGroups * kMaxStatBlocks));
-  c.stats = static_cast<float2*>(ar.take(sizeof(float2) * kMaxGroups));
+  c.gn_acc = h ? reinterpret_cast<unsigned long long*>(h + kHeaderBytes) : nullptr;
+  c.gn_seq = nullptr;
   c.skws = static_cast<float*>(ar.take(kSplitKBytes));
   c.skws_bytes = kSplitKBytes;
   c.st = st;
@@ -119,15 +119,10 @@ int run_gemv(const Ctx& c, const sdk::GemvBatch& b) {
 // GroupNorm (+SiLU) of [x0 | x1] into y.
 sd_status run_gn(const Ctx& c, const bf16* x0, int C0, const bf16* x1, int C1, int HW, int G, float eps,
                  const bf16* gamma, const bf16* beta, int silu, bf16* y) {
-  const double bytes = (double)HW * (C0 + C1) * 2;
-  {
-    sdp::Scope sc("gn_stats", sdp::F_GN_STATS, 0, bytes, c.st);
-    CK(sdk::launch_gn_stats(x0, C0, x1, C1, HW, G, eps, c.partial, c.counter, c.stats, c.sms, c.st));
-  }
-  {
-    sdp::Scope sc("gn_apply", sdp::F_GN_APPLY, 0, 2 * bytes, c.st);
-    CK(sdk::launch_gn_apply(x0, C0, x1, C1, HW, G, c.stats, gamma, beta, silu, y, c.sms, c.st));
-  }
+  if (!c.gn_seq || *c.gn_seq >= kMaxGnLaunches) return SD_ERR_UNSUPPORTED;
+  unsigned long long* acc = c.gn_acc + (size_t)(*c.gn_seq)++ * 2 * kMaxGroups;
+  sdp::Scope sc("groupnorm", sdp::F_GN_APPLY, 0, 3.0 * HW * (C0 + C1) * 2, c.st, 2);
+  CK(sdk::launch_groupnorm(x0, C0, x1, C1, HW, G, eps, gamma, beta, silu, y, acc, c.sms, c.st));
   return SD_OK;
 }
 
@@ -175,7 +170,7 @@ void add_conv3x3_segs(GemmProblem& p, int amap, int bmap, int C) {
 // y[M, N] = A[M, K] B[N, K]^T (+ epilogue), A a token matrix.
 sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, int N, const bf16* bias,
                      const bf16* residual, int ld_res, bf16* out, int ld_out, int mode = sdk::GEMM_PLAIN,
-                     double alg_k = 0) {
+                     double alg_k = 0, int f16_begin = 0) {
   GemmProblem p = base_problem(c);
   p.Ho = 1;
   p.Wo = M;
@@ -192,6 +187,7 @@ sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, i
   p.epi.out = out;
   p.epi.ld_out = ld_out;
   p.epi.mode = mode;
+  p.epi.f16_begin = f16_begin;
   CK(launch_gemm(c, p, alg_k));
   return SD_OK;
 }
@@ -674,8 +670,9 @@ sd_status check_ws(size_t need, const void* ws, size_t ws_bytes) {
   return SD_OK;
 }
 
+// Zero the device error word and this call's GroupNorm accumulators.
 sd_status clear_header(const Ctx& c) {
-  if (cudaMemsetAsync(c.err, 0, 8, c.st) != cudaSuccess) return SD_ERR_LAUNCH;
+  if (cudaMemsetAsync(c.err, 0, kHeaderBytes + kGnAccBytes, c.st) != cudaSuccess) return SD_ERR_LAUNCH;
   return SD_OK;
 }
 
@@ -853,6 +850,8 @@ sd_status sd_time_embed(const sd_time_cfg* cfg, const void* pw, float timestep, 
   TimePlan p;
   plan_time(a, cfg, (cudaStream_t)stream, d.sms, &p);
   if ((s = clear_header(p.c)) != SD_OK) return s;
+  int gn_seq = 0;
+  p.c.gn_seq = &gn_seq;
   Table tab;
   TimeW w = add_time(tab, "time", cfg->proj_dim, cfg->temb_dim);
   return run_time(p.c, w, pw, cfg->proj_dim, cfg->temb_dim, timestep, p.phi, p.hid, temb);
@@ -874,6 +873,8 @@ sd_status sd_conv_fwd(const sd_conv_cfg* cfg, int32_t kind, const void* pw, cons
   ConvPlan p;
   plan_conv(a, cfg, kind, (cudaStream_t)stream, d.sms, &p);
   if ((s = clear_header(p.c)) != SD_OK) return s;
+  int gn_seq = 0;
+  p.c.gn_seq = &gn_seq;
   Table tab;
   const int H = cfg->height, Wd = cfg->width;
   const bf16* X0 = static_cast<const bf16*>(x0);
@@ -916,6 +917,8 @@ sd_status sd_resblock_fwd(const sd_resblock_cfg* cfg, const void* pw, const void
   ResPlan p;
   plan_res(a, cfg, (cudaStream_t)stream, d.sms, &p);
   if ((s = clear_header(p.c)) != SD_OK) return s;
+  int gn_seq = 0;
+  p.c.gn_seq = &gn_seq;
   Table tab;
   ResW w = add_resblock(tab, "res", cfg->c_x + cfg->c_skip, cfg->c_out, cfg->temb_dim);
   sdk::GemvBatch b;
@@ -944,6 +947,8 @@ sd_status sd_transformer_fwd(const sd_transformer_cfg* cfg, const void* pw, cons
   TxPlan p;
   plan_tx(a, cfg, (cudaStream_t)stream, d.sms, &p);
   if ((s = clear_header(p.c)) != SD_OK) return s;
+  int gn_seq = 0;
+  p.c.gn_seq = &gn_seq;
   Table tab;
   TxW w = add_transformer(tab, "attn", cfg->channels, cfg->depth, cfg->ctx_dim);
   return run_transformer(p.c, w, pw, cfg->height, cfg->width, static_cast<const bf16*>(x),
@@ -965,6 +970,8 @@ sd_status sd_unet_step(const sd_unet_cfg* cfg, const void* pw, const void* laten
   plan_unet(a, cfg, (cudaStream_t)stream, d.sms, &p);
   const Ctx& c = p.c;
   if ((s = clear_header(c)) != SD_OK) return s;
+  int gn_seq = 0;
+  p.c.gn_seq = &gn_seq;
   Table tab;
   UNetW u = add_unet(tab, *cfg);
   const int L = cfg->n_levels;

@@ -58,6 +58,15 @@ __device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t smem_addr) {
   return d;
 }
 
+// BF16 pair by integer rounding (half away from zero in magnitude) on the ALU
+// pipe, leaving the conversion unit free for the exponentials; inputs are
+// finite and non-negative here.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u;
+  const uint32_t b = __float_as_uint(hi) + 0x8000u;
+  return __byte_perm(a, b, 0x7632);
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -282,7 +291,7 @@ __global__ void __launch_bounds__(192, 2)
           const float p0 = ex2(fmaf(__uint_as_float(sv[c * 32 + 2 * i]), sl2, -m_used));
           const float p1 = ex2(fmaf(__uint_as_float(sv[c * 32 + 2 * i + 1]), sl2, -m_used));
           l += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          pk[i] = pack_bf16x2_alu(p0, p1);
         }
         // keys c*32 .. c*32+31 = half c/2, 16-byte chunks 4*(c&1) .. +3, swizzled by row
         uint8_t* hrow = prow0 + (c >> 1) * kTileBytes;

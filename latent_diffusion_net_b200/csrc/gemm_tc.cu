@@ -236,7 +236,14 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       __nv_bfloat16* dst = args.epi.out + grow * args.epi.ld_out + nb;
-      if (full) {
+      if (full && args.epi.f16_begin > 0 && nb >= args.epi.f16_begin) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          d4[u] = make_uint4(pack_f16x2(v[8 * u + 0], v[8 * u + 1]), pack_f16x2(v[8 * u + 2], v[8 * u + 3]),
+                             pack_f16x2(v[8 * u + 4], v[8 * u + 5]), pack_f16x2(v[8 * u + 6], v[8 * u + 7]));
+        }
+      } else if (full) {
         uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -296,8 +303,12 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int spli
       v[0] += bf16lo(r.x); v[1] += bf16hi(r.x); v[2] += bf16lo(r.y); v[3] += bf16hi(r.y);
       v[4] += bf16lo(r.z); v[5] += bf16hi(r.z); v[6] += bf16lo(r.w); v[7] += bf16hi(r.w);
     }
-    *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) =
-        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    if (epi.f16_begin > 0 && c >= epi.f16_begin)
+      *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) =
+          make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
+    else
+      *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) =
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
   }
 }
 

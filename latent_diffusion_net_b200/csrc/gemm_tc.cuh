@@ -47,6 +47,7 @@ struct GemmEpi {
   __nv_bfloat16* out;             // [M][ld_out]
   int32_t ld_out;
   int32_t mode;                   // GemmMode
+  int32_t f16_begin;              // > 0: output columns >= f16_begin are stored as FP16 (a multiple of 32)
 };
 
 // A full problem: output grid Ho x Wo (M = Ho*Wo rows), N output features.

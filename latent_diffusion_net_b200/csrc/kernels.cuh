@@ -7,15 +7,12 @@
 
 namespace sdk {
 
-// GroupNorm: statistics over the channel concatenation [x0 | x1] (x1 may be
-// null with C1 = 0); `partial` holds gn_stats_blocks() * G float2 values and
-// `counter` one zero-initialised word (left at zero on return).
-int gn_stats_blocks(int HW, int C, int num_sms);
-int launch_gn_stats(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G, float eps,
-                    float2* partial, unsigned int* counter, float2* stats, int num_sms, cudaStream_t st);
-int launch_gn_apply(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G,
-                    const float2* stats, const __nv_bfloat16* gamma, const __nv_bfloat16* beta, int silu,
-                    __nv_bfloat16* y, int num_sms, cudaStream_t st);
+// GroupNorm (+SiLU) of the channel concatenation [x0 | x1] (x1 may be null with
+// C1 = 0) into y: a statistics kernel and an apply kernel. `acc` holds 2*G
+// zero-initialised 64-bit words used by this call only.
+int launch_groupnorm(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G, float eps,
+                     const __nv_bfloat16* gamma, const __nv_bfloat16* beta, int silu, __nv_bfloat16* y,
+                     unsigned long long* acc, int num_sms, cudaStream_t st);
 int launch_layernorm(const __nv_bfloat16* x, int N, int C, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,
                      float eps, __nv_bfloat16* y, cudaStream_t st);
 
