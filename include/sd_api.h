@@ -286,6 +286,19 @@ sd_status sd_profile_begin(void);
 sd_status sd_profile_end(int32_t* n_kernels); /* kernels enqueued while recording */
 sd_status sd_profile_read(sd_launch_record* out, int32_t capacity, int32_t* n);
 
+/* Tuning and test hook for the tensor-core GEMM behind every convolution and
+ * linear layer. bn (0 = automatic, else one of 32, 64, 96, 128, 160, 192, 224,
+ * 256) fixes the output-feature width of a tile; splits (0 = automatic, 1 = no
+ * split, up to 16) fixes the number of reduction splits. The setting is
+ * process-wide and applies to calls issued after it. A split count above the
+ * number of 64-wide reduction blocks of a GEMM is lowered to that number; one
+ * that needs more FP32 workspace than the call has makes the call fail with
+ * SD_ERR_UNSUPPORTED. Results are
+ * the same for every setting up to FP32 summation order. Not thread-safe
+ * against calls in flight on other host threads. The pages have no
+ * counterpart: this only selects among equivalent schedules. */
+sd_status sd_gemm_override(int32_t bn, int32_t splits);
+
 /* Kernel launches issued by this library in this process so far. */
 int64_t sd_launch_count(void);
 

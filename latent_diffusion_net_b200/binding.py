@@ -106,6 +106,7 @@ _SIGS = {
     "sd_profile_end": (c_int32, [POINTER(c_int32)]),
     "sd_profile_read": (c_int32, [POINTER(sd_launch_record), c_int32, POINTER(c_int32)]),
     "sd_launch_count": (c_int64, []),
+    "sd_gemm_override": (c_int32, [c_int32, c_int32]),
 }
 
 _lib = None
@@ -315,6 +316,11 @@ def sd_profile_read():
 
 def sd_launch_count():
     return int(lib().sd_launch_count())
+
+
+def sd_gemm_override(bn=0, splits=0):
+    """Fix the GEMM N tile and reduction split count (0 = automatic)."""
+    _check(lib().sd_gemm_override(int(bn), int(splits)), "sd_gemm_override")
 
 
 # ---------------------------------------------------------------- config helpers

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -98,6 +99,7 @@ Ctx make_ctx(Arena& ar, cudaStream_t st, int sms) {
 #define CK(x)                        \
   do {                               \
     int _e = (x);                    \
+    if (_e == -1) return SD_ERR_UNSUPPORTED; \
     if (_e != 0) return SD_ERR_LAUNCH; \
   } while (0)
 
@@ -129,7 +131,12 @@ sd_status run_gn(const Ctx& c, const bf16* x0, int C0, const bf16* x1, int C1, i
 // Launch a GEMM problem under a profiling scope with its algorithmic work:
 // FLOPs 2*M*N*K (K = reduction length; alg_k overrides a zero-padded K), bytes
 // = every A source and B matrix read once, the output (and residual) once.
-int launch_gemm(const Ctx& c, const GemmProblem& p, double alg_k = 0) {
+std::atomic<int> g_force_bn{0}, g_force_splits{0};
+
+int launch_gemm(const Ctx& c, const GemmProblem& p0, double alg_k = 0) {
+  GemmProblem p = p0;
+  p.force_bn = g_force_bn.load(std::memory_order_relaxed);
+  p.force_splits = g_force_splits.load(std::memory_order_relaxed);
   double K = 0;
   for (int i = 0; i < p.nseg; ++i) K += 64.0 * p.seg[i].nkb;
   if (alg_k > 0) K = alg_k;
@@ -682,6 +689,14 @@ sd_status clear_header(const Ctx& c) {
 extern "C" {
 
 const char* sd_version(void) { return "sd-b200 0.1"; }
+
+sd_status sd_gemm_override(int32_t bn, int32_t splits) {
+  const bool bn_ok = bn == 0 || (bn >= 32 && bn <= 256 && bn % 32 == 0);
+  if (!bn_ok || splits < 0 || splits > 16) return SD_ERR_UNSUPPORTED;
+  g_force_bn.store(bn, std::memory_order_relaxed);
+  g_force_splits.store(splits, std::memory_order_relaxed);
+  return SD_OK;
+}
 
 const char* sd_status_string(sd_status s) {
   switch (s) {

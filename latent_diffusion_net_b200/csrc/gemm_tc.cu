@@ -1,17 +1,17 @@
 // tcgen05 implicit GEMM for sm_100a.
 //
 // D[M, N] = sum over K-segments of A_seg[M, 64*nkb] * B_seg[N, 64*nkb]^T, then
-// epilogue: + bias + bias2 + colvec, + residual, BF16 store (or GEGLU pairs).
+// epilogue: + bias + bias2 + colvec, + residual, BF16 store (or GEGLU pairs),
+// or FP32 partial sums for a split reduction.
 //
-// Roles (192 threads): warp 0 lane 0 issues TMA loads of A (4-D box of a
-// BHxBW pixel rectangle x 64 channels, zero-filled outside the image, which is
-// exactly the zero padding of a 3x3 convolution) and B (64 x BN weight tile);
-// warp 1 owns the TMEM accumulator and lane 0 issues tcgen05.mma (M=128, N=BN,
-// K=16, BF16 in, FP32 accumulate); warps 2..5 are the epilogue, one TMEM lane
-// quarter each (warp w reads lanes 32*(w%4) .. +31).
+// A operand: a 4-D TMA box of a BHxBW pixel rectangle x 64 channels, zero-
+// filled outside the image, which is exactly the zero padding of a 3x3
+// convolution; each 3x3 tap is one K-segment with the box shifted by (dx, dy).
+// B operand: 64-wide K slices of the [N][K] weight matrix.
 #include "common.cuh"
 #include "gemm_tc.cuh"
 
+#include <algorithm>
 #include <mutex>
 
 namespace sdk {
@@ -19,6 +19,8 @@ namespace sdk {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
+constexpr int kEpiThreads = 256;              // 8 epilogue warps, two per TMEM lane quarter
+constexpr int kGemmThreads = 64 + kEpiThreads;
 
 struct __align__(64) GemmMaps {
   CUtensorMap a[kGemmMaxA];
@@ -26,59 +28,134 @@ struct __align__(64) GemmMaps {
 };
 
 struct GemmArgs {
-  int32_t Ho, Wo, BH, BW, tiles_x, N;
+  int32_t Ho, Wo, BH, BW, tiles_x, tiles_m, N;
   int32_t nseg, total_kb;
-  int32_t kb_per_split;  // k-blocks per blockIdx.z (== total_kb without split-K)
+  int32_t kb_per_split, splits, tiles_n, units;
   GemmSeg seg[kGemmMaxSeg];
   GemmEpi epi;
-  float* partial;  // split-K: FP32 [gridDim.z][Ho*Wo][N]; null otherwise
+  float* partial;  // split-K: FP32 [splits][Ho*Wo][N]; null otherwise
   int* err;
-};
-
-template <int BN>
-struct TmemCols {
-  static constexpr uint32_t value = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
 };
 
 __device__ __forceinline__ float gelu_erf(float g) { return 0.5f * g * (1.0f + erff(g * 0.70710678118654752f)); }
 
+// ------------------------------------------------------------------ 2-SM helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared-memory address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA loads of a CTA pair: the data lands in this CTA's shared memory, the
+// transaction bytes are counted on the barrier of the even CTA of the pair.
+constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;
+__device__ __forceinline__ void tma2_load_2d(void* dst, const void* tmap, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar) & kPeerBitMask), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma2_load_4d(void* dst, const void* tmap, uint64_t* bar, int c0, int c1, int c2,
+                                             int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, "
+      "%5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar) & kPeerBitMask), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_2sm(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_2sm(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem] (+)= A[smem of both CTAs] * B[smem of both CTAs]^T, M = 256, issued by the even CTA.
+__device__ __forceinline__ void umma2_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` in both CTAs of the pair once the issued MMAs complete.
+__device__ __forceinline__ void umma2_commit_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)0x3)
+      : "memory");
+}
+
+// ------------------------------------------------------------------ the kernel
+// A cluster of two CTAs (one per SM) computes 256 x BN output tiles with
+// tcgen05.mma.cta_group::2: each CTA loads the 128 rows of A of its own
+// 128-pixel tile and BN/2 rows of B; the even CTA issues the MMAs, which read
+// both CTAs' shared memory and write each CTA's half of the accumulator into its
+// own TMEM. The cluster walks a static list of work units (pair of M tiles, N
+// tile, K split); accumulators are double-buffered in TMEM so the epilogue of
+// one unit overlaps the main loop of the next.
+// Roles (320 threads per CTA): warp 0 lane 0 TMA producer (both CTAs); warp 1
+// owns TMEM, lane 0 of the even CTA issues MMAs; warps 2-9 epilogue (TMEM lane
+// quarter warp % 4; warps 2-5 take the even 32-column chunks, 6-9 the odd ones).
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args) {
-  constexpr int kBTileBytes = BN * kBK * 2;
-  constexpr int kStageBytes = kATileBytes + kBTileBytes;
-  constexpr uint32_t kTmemCols = TmemCols<BN>::value;
-  constexpr uint32_t kIdesc = umma_idesc_bf16(kBM, BN);
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "epilogue works in 32-column chunks");
+  constexpr int kBHalf = BN / 2;
+  constexpr int kBTileBytes = kBHalf * kBK * 2;
+  constexpr int kStageBytes = kATileBytes + kBTileBytes;
+  constexpr uint32_t kTmemCols = 512;  // two accumulators of up to 256 columns
+  constexpr uint32_t kIdesc = umma_idesc_bf16(256, BN);
+  constexpr int kChunks = BN / 32;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
   uint64_t* empty_bar = full_bar + STAGES;
-  uint64_t* accum_bar = empty_bar + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_bar + 1);
+  uint64_t* acc_full = empty_bar + STAGES;  // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2], used in the even CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* epi_col = reinterpret_cast<float*>(tmem_slot + 4);  // [BN]
+  float* epi_col = reinterpret_cast<float*>(smem + STAGES * kStageBytes + 256);  // [2][256]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int mt = blockIdx.x;
-  const int n0 = blockIdx.y * BN;
-  const int tile_y0 = (mt / args.tiles_x) * args.BH;
-  const int tile_x0 = (mt % args.tiles_x) * args.BW;
+  const uint32_t rank = cluster_rank();
+  const int cluster_id = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    mbar_init(accum_bar, 1);
+    mbar_init(&acc_full[0], 1);
+    mbar_init(&acc_full[1], 1);
+    mbar_init(&acc_empty[0], 2);
+    mbar_init(&acc_empty[1], 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 1) tmem_alloc_2sm(tmem_slot, kTmemCols);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // everything above touched only shared memory and TMEM: wait for the previous kernel here
@@ -90,178 +167,248 @@ __global__ void __launch_bounds__(192, 1)
       for (int i = 0; i < kGemmMaxA; ++i) tma_prefetch_desc(&maps.a[i]);
       tma_prefetch_desc(&maps.b[0]);
       tma_prefetch_desc(&maps.b[1]);
-      const int kb_lo = blockIdx.z * args.kb_per_split;
-      const int kb_hi = min(args.total_kb, kb_lo + args.kb_per_split);
-      int g = 0;  // position in the whole reduction
+      uint32_t q = 0;  // k-blocks issued by this CTA so far (stage ring position)
       bool ok = true;
-      for (int si = 0; si < args.nseg && ok && g < kb_hi; ++si) {
-        const GemmSeg sg = args.seg[si];
-        for (int j = 0; j < sg.nkb; ++j, ++g) {
-          if (g < kb_lo) continue;
-          if (g >= kb_hi) break;
-          const int kb = g - kb_lo;
-          const int s = kb % STAGES;
-          const int it = kb / STAGES;
-          if (kb >= STAGES && !mbar_wait(&empty_bar[s], (it - 1) & 1, abort_flag, args.err)) {
-            ok = false;
-            break;
+      for (int u = cluster_id; u < args.units && ok; u += nclusters) {
+        const int z = u % args.splits;
+        const int rest = u / args.splits;
+        const int nt = rest % args.tiles_n;
+        const int mt = (rest / args.tiles_n) * 2 + (int)rank;
+        const int tile_y0 = (mt / args.tiles_x) * args.BH;  // past the image for a dummy tile: zero fill
+        const int tile_x0 = (mt % args.tiles_x) * args.BW;
+        const int brow = nt * BN + (int)rank * kBHalf;
+        const int kb_lo = z * args.kb_per_split;
+        const int kb_hi = min(args.total_kb, kb_lo + args.kb_per_split);
+        int g = 0;
+        for (int si = 0; si < args.nseg && ok && g < kb_hi; ++si) {
+          const GemmSeg sg = args.seg[si];
+          for (int j = 0; j < sg.nkb; ++j, ++g) {
+            if (g < kb_lo) continue;
+            if (g >= kb_hi) break;
+            const uint32_t s = q % STAGES;
+            if (q >= (uint32_t)STAGES && !mbar_wait(&empty_bar[s], ((q / STAGES) - 1) & 1, abort_flag, args.err)) {
+              ok = false;
+              break;
+            }
+            uint8_t* a_dst = smem + s * kStageBytes;
+            uint8_t* b_dst = a_dst + kATileBytes;
+            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * kStageBytes);
+            tma2_load_4d(a_dst, &maps.a[sg.amap], &full_bar[s], sg.c0 + j * kBK, tile_x0 + sg.dx, tile_y0 + sg.dy,
+                         sg.z);
+            tma2_load_2d(b_dst, &maps.b[sg.bmap], &full_bar[s], sg.bk0 + j * kBK, brow);
+            ++q;
           }
-          uint8_t* a_dst = smem + s * kStageBytes;
-          uint8_t* b_dst = a_dst + kATileBytes;
-          mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
-          tma_load_4d(a_dst, &maps.a[sg.amap], &full_bar[s], sg.c0 + j * kBK, tile_x0 + sg.dx, tile_y0 + sg.dy,
-                      sg.z);
-          tma_load_2d(b_dst, &maps.b[sg.bmap], &full_bar[s], sg.bk0 + j * kBK, n0);
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
+      uint32_t q = 0;
+      int it = 0;
       bool ok = true;
-      const int kb_lo = blockIdx.z * args.kb_per_split;
-      const int nkb = min(args.total_kb, kb_lo + args.kb_per_split) - kb_lo;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % STAGES;
-        const int it = kb / STAGES;
-        if (!mbar_wait(&full_bar[s], it & 1, abort_flag, args.err)) {
-          ok = false;
-          break;
-        }
+      for (int u = cluster_id; u < args.units && ok; u += nclusters, ++it) {
+        const int z = u % args.splits;
+        const int kb_lo = z * args.kb_per_split;
+        const int nkb = min(args.total_kb, kb_lo + args.kb_per_split) - kb_lo;
+        const int b = it & 1;
+        // the epilogues of both CTAs must have drained this accumulator (first use passes)
+        if (!mbar_wait(&acc_empty[b], ((it >> 1) & 1) ^ 1, abort_flag, args.err)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
-        const uint32_t b_addr = a_addr + kATileBytes;
-        const uint64_t adesc = umma_desc_k_sw128(a_addr);
-        const uint64_t bdesc = umma_desc_k_sw128(b_addr);
+        const uint32_t tacc = tmem_base + (uint32_t)(b * 256);
+        for (int kb = 0; kb < nkb; ++kb, ++q) {
+          const uint32_t s = q % STAGES;
+          if (!mbar_wait(&full_bar[s], (q / STAGES) & 1, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+          const uint64_t adesc = umma_desc_k_sw128(a_addr);
+          const uint64_t bdesc = umma_desc_k_sw128(a_addr + kATileBytes);
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          // +32 bytes along K inside the 128-byte swizzle row = +2 in the encoded address
-          umma_bf16(tmem_base, adesc + 2 * k, bdesc + 2 * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < kBK / 16; ++k) {
+            // +32 bytes along K inside the 128-byte swizzle row = +2 in the encoded address
+            umma2_bf16(tacc, adesc + 2 * k, bdesc + 2 * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma2_commit_both(&empty_bar[s]);
         }
-        umma_commit(&empty_bar[s]);
+        if (ok) umma2_commit_both(&acc_full[b]);
       }
-      if (ok) umma_commit(accum_bar);
     }
   } else {
-    // ---------------------------------------------------------------- epilogue
-    const int et = threadIdx.x - 64;  // 0..127
-    for (int c = et; c < BN; c += 128) {
-      const int n = n0 + c;
-      float v = 0.f;
-      if (n < args.N && !args.partial) {
-        if (args.epi.bias) v += __bfloat162float(args.epi.bias[n]);
-        if (args.epi.bias2) v += __bfloat162float(args.epi.bias2[n]);
-        if (args.epi.colvec) v += args.epi.colvec[n];
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    // Every argument the loop needs is copied to registers once: reads of the
+    // kernel parameters inside the unrolled loops cannot be hoisted past the
+    // global stores by the compiler and would be repeated per element.
+    const int N = args.N, Ho = args.Ho, Wo = args.Wo, BH = args.BH, BW = args.BW;
+    const int tiles_x = args.tiles_x, tiles_m = args.tiles_m, tiles_n = args.tiles_n, splits = args.splits;
+    const int units = args.units;
+    float* const partial = args.partial;
+    const __nv_bfloat16* const bias = args.epi.bias;
+    const __nv_bfloat16* const bias2 = args.epi.bias2;
+    const float* const colvec = args.epi.colvec;
+    const __nv_bfloat16* const residual = args.epi.residual;
+    const int ld_res = args.epi.ld_res, ld_out = args.epi.ld_out, f16_begin = args.epi.f16_begin;
+    const bool geglu = args.epi.mode == GEMM_GEGLU;
+    __nv_bfloat16* const out = args.epi.out;
+    const bool has_cols = partial == nullptr && (bias || bias2 || colvec);
+
+    const int et = threadIdx.x - 64;  // 0..255
+    const int half = (warp - 2) >> 2;  // which alternate 32-column chunks this warp handles
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t leader_empty0 = map_to_rank(smem_u32(&acc_empty[0]), 0);
+    const uint32_t leader_empty1 = map_to_rank(smem_u32(&acc_empty[1]), 0);
+    int it = 0;
+    for (int u = cluster_id; u < units; u += nclusters, ++it) {
+      const int z = u % splits;
+      const int rest = u / splits;
+      const int nt = rest % tiles_n;
+      const int mt = (rest / tiles_n) * 2 + (int)rank;
+      const int n0 = nt * BN;
+      const int b = it & 1;
+      float* const ecol = epi_col + b * 256;
+      if (has_cols) {
+        // per-column terms of this unit (biases + FP32 column vector), computed
+        // while the main loop runs; buffer b was last read two units ago
+        for (int c = et; c < BN; c += kEpiThreads) {
+          const int n = n0 + c;
+          float a = 0.f;
+          if (n < N) {
+            if (bias) a += __bfloat162float(bias[n]);
+            if (bias2) a += __bfloat162float(bias2[n]);
+            if (colvec) a += colvec[n];
+          }
+          ecol[c] = a;
+        }
+        asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
       }
-      epi_col[c] = v;
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    const bool have = mbar_wait(accum_bar, 0, abort_flag, args.err);
-    tc_fence_after();
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const int oy = tile_y0 + row / args.BW;
-    const int ox = tile_x0 + row % args.BW;
-    const bool valid = have && oy < args.Ho && ox < args.Wo;
-    const long grow = (long)oy * args.Wo + ox;
+      const bool have = mbar_wait(&acc_full[b], (it >> 1) & 1, abort_flag, args.err);
+      tc_fence_after();
+      const int oy = (mt / tiles_x) * BH + row / BW;
+      const int ox = (mt % tiles_x) * BW + row % BW;
+      const bool valid = have && mt < tiles_m && oy < Ho && ox < Wo;
+      const long grow = (long)oy * Wo + ox;
+      const uint32_t tacc = tmem_base + (uint32_t)(b * 256) + lane_off;
+      if (half >= kChunks) {
+        // no chunk for this warp (BN = 32): still take part in the release
+        tc_fence_before();
+        asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+      }
 #pragma unroll 1
-    for (int cc = 0; cc < BN / 32; ++cc) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + cc * 32, r);
-      tmem_ld_wait();
-      if (!valid) continue;
-      const int nb = n0 + cc * 32;
-      if (nb >= args.N) continue;
-      float v[32];
+      for (int cc = half; cc < kChunks; cc += 2) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tacc + cc * 32, r);
+        tmem_ld_wait();
+        if (cc + 2 >= kChunks) {
+          // this warp's last read of the accumulator: once all epilogue warps
+          // are here it goes back to the MMA issuer
+          tc_fence_before();
+          asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+          if (warp == 2 && lane == 0) mbar_arrive_cluster(b ? leader_empty1 : leader_empty0);
+        }
+        if (!valid) continue;
+        const int nb = n0 + cc * 32;
+        if (nb >= N) continue;
+        float v[32];
+        if (has_cols) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + epi_col[cc * 32 + j];
-      const bool full = (nb + 32 <= args.N);
-      if (args.partial) {
-        float* dst = args.partial + ((size_t)blockIdx.z * args.Ho * args.Wo + grow) * args.N + nb;
-        if (full) {
-          float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) d4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + ecol[cc * 32 + j];
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (nb + j < args.N) dst[j] = v[j];
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
         }
-        continue;
-      }
-      if (args.epi.mode == GEMM_GEGLU) {
-        // columns (2j, 2j+1) hold (value_j, gate_j); output column (nb/2 + j)
-        uint32_t o[8];
+        const bool full = (nb + 32 <= N);
+        if (partial) {
+          float* dst = partial + ((size_t)z * Ho * Wo + grow) * N + nb;
+          if (full) {
+            float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float a0 = v[4 * j] * gelu_erf(v[4 * j + 1]);
-          const float a1 = v[4 * j + 2] * gelu_erf(v[4 * j + 3]);
-          o[j] = pack_bf16x2(a0, a1);
+            for (int w = 0; w < 8; ++w) d4[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (nb + j < N) dst[j] = v[j];
+          }
+          continue;
         }
-        __nv_bfloat16* dst = args.epi.out + grow * args.epi.ld_out + (nb >> 1);
-        if (full) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
-          d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
-          d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
-        } else {
+        if (geglu) {
+          // columns (2j, 2j+1) hold (value_j, gate_j); output column (nb/2 + j)
+          uint32_t o[8];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (nb + 2 * j < args.N) {
-              const uint32_t w = o[j >> 1];
-              dst[j] = __ushort_as_bfloat16((unsigned short)((j & 1) ? (w >> 16) : (w & 0xFFFF)));
+          for (int j = 0; j < 8; ++j) {
+            const float a0 = v[4 * j] * gelu_erf(v[4 * j + 1]);
+            const float a1 = v[4 * j + 2] * gelu_erf(v[4 * j + 3]);
+            o[j] = pack_bf16x2(a0, a1);
+          }
+          __nv_bfloat16* dst = out + grow * ld_out + (nb >> 1);
+          if (full) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+            d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (nb + 2 * j < N) {
+                const uint32_t w = o[j >> 1];
+                dst[j] = __ushort_as_bfloat16((unsigned short)((j & 1) ? (w >> 16) : (w & 0xFFFF)));
+              }
             }
           }
+          continue;
         }
-        continue;
-      }
-      if (args.epi.residual) {
-        const __nv_bfloat16* rs = args.epi.residual + grow * args.epi.ld_res + nb;
-        if (full) {
-          const uint4* r4 = reinterpret_cast<const uint4*>(rs);
+        if (residual) {
+          const __nv_bfloat16* rs = residual + grow * ld_res + nb;
+          if (full) {
+            const uint4* r4 = reinterpret_cast<const uint4*>(rs);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 w = r4[u];
-            v[8 * u + 0] += bf16lo(w.x);
-            v[8 * u + 1] += bf16hi(w.x);
-            v[8 * u + 2] += bf16lo(w.y);
-            v[8 * u + 3] += bf16hi(w.y);
-            v[8 * u + 4] += bf16lo(w.z);
-            v[8 * u + 5] += bf16hi(w.z);
-            v[8 * u + 6] += bf16lo(w.w);
-            v[8 * u + 7] += bf16hi(w.w);
+            for (int w4 = 0; w4 < 4; ++w4) {
+              const uint4 w = r4[w4];
+              v[8 * w4 + 0] += bf16lo(w.x);
+              v[8 * w4 + 1] += bf16hi(w.x);
+              v[8 * w4 + 2] += bf16lo(w.y);
+              v[8 * w4 + 3] += bf16hi(w.y);
+              v[8 * w4 + 4] += bf16lo(w.z);
+              v[8 * w4 + 5] += bf16hi(w.z);
+              v[8 * w4 + 6] += bf16lo(w.w);
+              v[8 * w4 + 7] += bf16hi(w.w);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (nb + j < N) v[j] += __bfloat162float(rs[j]);
+          }
+        }
+        __nv_bfloat16* dst = out + grow * ld_out + nb;
+        if (full && f16_begin > 0 && nb >= f16_begin) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            d4[w] = make_uint4(pack_f16x2(v[8 * w + 0], v[8 * w + 1]), pack_f16x2(v[8 * w + 2], v[8 * w + 3]),
+                               pack_f16x2(v[8 * w + 4], v[8 * w + 5]), pack_f16x2(v[8 * w + 6], v[8 * w + 7]));
+          }
+        } else if (full) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            d4[w] = make_uint4(pack_bf16x2(v[8 * w + 0], v[8 * w + 1]), pack_bf16x2(v[8 * w + 2], v[8 * w + 3]),
+                               pack_bf16x2(v[8 * w + 4], v[8 * w + 5]), pack_bf16x2(v[8 * w + 6], v[8 * w + 7]));
           }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (nb + j < args.N) v[j] += __bfloat162float(rs[j]);
+            if (nb + j < N) dst[j] = __float2bfloat16_rn(v[j]);
         }
-      }
-      __nv_bfloat16* dst = args.epi.out + grow * args.epi.ld_out + nb;
-      if (full && args.epi.f16_begin > 0 && nb >= args.epi.f16_begin) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          d4[u] = make_uint4(pack_f16x2(v[8 * u + 0], v[8 * u + 1]), pack_f16x2(v[8 * u + 2], v[8 * u + 3]),
-                             pack_f16x2(v[8 * u + 4], v[8 * u + 5]), pack_f16x2(v[8 * u + 6], v[8 * u + 7]));
-        }
-      } else if (full) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          d4[u] = make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
-                             pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (nb + j < args.N) dst[j] = __float2bfloat16_rn(v[j]);
       }
     }
   }
 
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+  if (warp == 1) tmem_dealloc_2sm(tmem_base, kTmemCols);
 }
 
 // Split-K reduction: out = epilogue(sum over splits of partial), 8 columns per
@@ -360,11 +507,16 @@ bool tmap_encode_4d(CUtensorMap* m, const void* ptr, const uint64_t d[4], uint32
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES>
-static int launch_bn(const GemmMaps& maps, const GemmArgs& args, int tiles_m, int tiles_n, int splits,
-                     cudaStream_t st) {
-  constexpr int kStageBytes = kATileBytes + BN * kBK * 2;
-  constexpr size_t smem = 1024 + (size_t)STAGES * kStageBytes + 256 + BN * 4;
+template <int BN>
+struct Stages {
+  static constexpr int value = (kATileBytes + BN * kBK) * 8 <= 200 * 1024 ? 8 : 6;
+};
+
+template <int BN>
+static int launch_bn(const GemmMaps& maps, const GemmArgs& args, int grid, cudaStream_t st) {
+  constexpr int STAGES = Stages<BN>::value;
+  constexpr int kStageBytes = kATileBytes + (BN / 2) * kBK * 2;
+  constexpr size_t smem = 1024 + (size_t)STAGES * kStageBytes + 256 + 2048;
   static bool attr_set = false;  // benign race: the attribute value is identical for every caller
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -372,7 +524,7 @@ static int launch_bn(const GemmMaps& maps, const GemmArgs& args, int tiles_m, in
     if (e != cudaSuccess) return (int)e;
     attr_set = true;
   }
-  return (int)launch_pdl(gemm_tc_kernel<BN, STAGES>, dim3(tiles_m, tiles_n, splits), dim3(192), smem, st, maps, args);
+  return (int)launch_pdl(gemm_tc_kernel<BN, STAGES>, dim3(grid), dim3(kGemmThreads), smem, st, maps, args);
 }
 
 static void choose_tile_rect(int Ho, int Wo, int* BH, int* BW) {
@@ -395,19 +547,8 @@ static void choose_tile_rect(int Ho, int Wo, int* BH, int* BW) {
   *BH = 128 / bw_best;
 }
 
-static int choose_bn(int N, int tiles_m, int num_sms) {
-  if (N <= 32) return 32;
-  const int cands[] = {256, 192, 160, 128, 64};
-  for (int bn : cands) {
-    if (N % bn) continue;
-    if ((long)tiles_m * (N / bn) >= (long)num_sms * 9 / 10) return bn;
-  }
-  if (N % 64 == 0) return 64;
-  return 0;
-}
-
 struct GemmPlan {
-  int BH, BW, tiles_x, tiles_m, bn, tiles_n, splits, kb_per_split, total_kb;
+  int BH, BW, tiles_x, tiles_m, bn, tiles_n, splits, kb_per_split, total_kb, units, clusters;
 };
 
 static int sm_count() {
@@ -421,37 +562,89 @@ static int sm_count() {
   return num_sms;
 }
 
+// CTA pairs that can be resident at once (a GPC with an odd number of SMs
+// leaves one SM out of every pairing).
+static int max_active_clusters() {
+  static int n = 0;
+  if (n == 0) {
+    constexpr int STAGES = Stages<256>::value;
+    constexpr size_t smem = 1024 + (size_t)STAGES * (kATileBytes + 128 * kBK * 2) + 256 + 2048;
+    cudaFuncSetAttribute(gemm_tc_kernel<256, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sm_count() / 2));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, gemm_tc_kernel<256, STAGES>, &cfg) != cudaSuccess || c <= 0) {
+      cudaGetLastError();
+      c = sm_count() / 2;
+    }
+    n = std::min(c, sm_count() / 2);
+  }
+  return n;
+}
+
+// Estimated cycles of a plan. Per k-block a CTA pair performs 2*256*BN*64 FLOPs
+// (2*BN cycles per SM at the tensor rate) and each SM loads 16 KB of A plus
+// BN*64 bytes of B (about 64 bytes per cycle per SM); the slower of the two
+// sets the pace. Units are spread over the clusters in rounds; the last
+// epilogue and the split-K reduction are added on top.
+static double plan_cost(int bn, int splits, int pairs, int N, int total_kb, long M, int clusters) {
+  const int tiles_n = (N + bn - 1) / bn;
+  const long units = (long)pairs * tiles_n * splits;
+  const long rounds = (units + clusters - 1) / clusters;
+  const int kb = (total_kb + splits - 1) / splits;
+  const double per_kb = std::max(2.0 * bn, 256.0 + bn);
+  double cost = (double)rounds * (kb * per_kb + 600.0) + 8.0 * bn;
+  if (splits > 1) cost += 4000.0 + (double)splits * M * N * 4.0 / 3000.0;
+  return cost;
+}
+
 // Tile shape, N tile and split-K factor for a problem.
 static bool plan_gemm(const GemmProblem& p, GemmPlan* g) {
-  const int sms = sm_count();
   choose_tile_rect(p.Ho, p.Wo, &g->BH, &g->BW);
   g->tiles_x = (p.Wo + g->BW - 1) / g->BW;
   g->tiles_m = g->tiles_x * ((p.Ho + g->BH - 1) / g->BH);
   g->total_kb = 0;
   for (int i = 0; i < p.nseg; ++i) g->total_kb += p.seg[i].nkb;
-  g->bn = p.force_bn ? p.force_bn : choose_bn(p.N, g->tiles_m, sms);
-  if (g->bn == 0 || g->total_kb <= 0) return false;
+  if (g->total_kb <= 0) return false;
+  const int pairs = (g->tiles_m + 1) / 2;
+  const int max_clusters = max_active_clusters();
+  const long M = (long)p.Ho * p.Wo;
+  const size_t per_split = (size_t)M * p.N * sizeof(float);
+  const int bns[] = {256, 224, 192, 160, 128, 96, 64, 32};
+  const int sps[] = {1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16};
+  double best = -1.0;
+  g->bn = 0;
   g->splits = 1;
-  // under-filled grid with a long reduction: a 128-wide N tile and split-K
-  const bool small = (long)g->tiles_m * (p.N / 64 > 0 ? p.N / 64 : 1) < sms && g->total_kb >= 16 && p.N % 128 == 0;
-  if (p.force_splits > 0) {
-    g->splits = p.force_splits;
-  } else if (small && p.splitk_ws && !p.force_bn) {
-    g->bn = 128;
-    const int ctas = g->tiles_m * (p.N / 128);
-    int sp = (sms + ctas - 1) / ctas;
-    if (sp > g->total_kb / 4) sp = g->total_kb / 4;
-    if (sp > 16) sp = 16;
-    const size_t per = (size_t)p.Ho * p.Wo * p.N * sizeof(float);
-    while (sp > 1 && per * sp > p.splitk_ws_bytes) --sp;
-    g->splits = sp < 1 ? 1 : sp;
+  for (int bn : bns) {
+    if (p.force_bn) {
+      if (bn != p.force_bn) continue;
+    } else {
+      if (bn > 32 && p.N <= bn / 2) continue;  // more than half the tile would be padding
+      if (bn == 32 && p.N > 64) continue;
+    }
+    for (int sp : sps) {
+      if (p.force_splits) {
+        if (sp != std::min(p.force_splits, g->total_kb)) continue;
+      } else if (sp > 1 && (g->total_kb / sp < 4 || (sp > 8 && sp % 2))) {
+        continue;
+      }
+      if (sp > 1 && (!p.splitk_ws || per_split * sp > p.splitk_ws_bytes || p.N % 8)) continue;
+      const double c = plan_cost(bn, sp, pairs, p.N, g->total_kb, M, max_clusters);
+      if (best < 0 || c < best) {
+        best = c;
+        g->bn = bn;
+        g->splits = sp;
+      }
+    }
   }
+  if (g->bn == 0) return false;
   g->tiles_n = (p.N + g->bn - 1) / g->bn;
   g->kb_per_split = (g->total_kb + g->splits - 1) / g->splits;
   g->splits = (g->total_kb + g->kb_per_split - 1) / g->kb_per_split;  // no empty split
-  if (g->splits > 1 && (!p.splitk_ws || (size_t)p.Ho * p.Wo * p.N * sizeof(float) * g->splits > p.splitk_ws_bytes ||
-                        p.N % 8))
-    return false;
+  g->units = pairs * g->tiles_n * g->splits;
+  g->clusters = std::min(g->units, max_clusters);
   return true;
 }
 
@@ -472,18 +665,19 @@ int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   args.BH = g.BH;
   args.BW = g.BW;
   args.tiles_x = g.tiles_x;
+  args.tiles_m = g.tiles_m;
   args.N = p.N;
   args.nseg = p.nseg;
   for (int i = 0; i < p.nseg; ++i) args.seg[i] = p.seg[i];
   args.total_kb = g.total_kb;
   args.kb_per_split = g.kb_per_split;
+  args.splits = g.splits;
+  args.tiles_n = g.tiles_n;
+  args.units = g.units;
   args.epi = p.epi;
   args.partial = g.splits > 1 ? p.splitk_ws : nullptr;
   args.err = p.err;
   const int bn = g.bn;
-  const int tiles_m = g.tiles_m;
-  const int tiles_n = g.tiles_n;
-  const int splits = g.splits;
 
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
@@ -494,25 +688,28 @@ int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   }
   for (int i = 0; i < kGemmMaxB; ++i) {
     const GemmBSrc& b = p.b[i < p.nb ? i : 0];
-    if (!tmap_encode_2d(&maps.b[i], b.ptr, (uint64_t)b.K, (uint64_t)b.rows, 64, (uint32_t)bn)) return -2;
+    if (!tmap_encode_2d(&maps.b[i], b.ptr, (uint64_t)b.K, (uint64_t)b.rows, 64, (uint32_t)(bn / 2))) return -2;
   }
+  const int grid = 2 * g.clusters;
   int e;
   switch (bn) {
-    case 32: e = launch_bn<32, 6>(maps, args, tiles_m, tiles_n, splits, stream); break;
-    case 64: e = launch_bn<64, 4>(maps, args, tiles_m, tiles_n, splits, stream); break;
-    case 128: e = launch_bn<128, 3>(maps, args, tiles_m, tiles_n, splits, stream); break;
-    case 160: e = launch_bn<160, 3>(maps, args, tiles_m, tiles_n, splits, stream); break;
-    case 192: e = launch_bn<192, 4>(maps, args, tiles_m, tiles_n, splits, stream); break;
-    case 256: e = launch_bn<256, 4>(maps, args, tiles_m, tiles_n, splits, stream); break;
+    case 32: e = launch_bn<32>(maps, args, grid, stream); break;
+    case 64: e = launch_bn<64>(maps, args, grid, stream); break;
+    case 96: e = launch_bn<96>(maps, args, grid, stream); break;
+    case 128: e = launch_bn<128>(maps, args, grid, stream); break;
+    case 160: e = launch_bn<160>(maps, args, grid, stream); break;
+    case 192: e = launch_bn<192>(maps, args, grid, stream); break;
+    case 224: e = launch_bn<224>(maps, args, grid, stream); break;
+    case 256: e = launch_bn<256>(maps, args, grid, stream); break;
     default: return -1;
   }
-  if (e != 0 || splits <= 1) return e;
+  if (e != 0 || g.splits <= 1) return e;
   const int M = p.Ho * p.Wo;
   const size_t vecs = (size_t)M * (p.N / 8);
   int blocks = (int)((vecs + 255) / 256);
   if (blocks > sm_count() * 8) blocks = sm_count() * 8;
-  return (int)launch_pdl(splitk_reduce_kernel, dim3(blocks), dim3(256), 0, stream, (const float*)p.splitk_ws, splits, M,
-                         p.N, p.epi);
+  return (int)launch_pdl(splitk_reduce_kernel, dim3(blocks), dim3(256), 0, stream, (const float*)p.splitk_ws,
+                         g.splits, M, p.N, p.epi);
 }
 
 }  // namespace sdk

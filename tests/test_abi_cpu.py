@@ -170,3 +170,12 @@ def test_workspace_sizes():
     large = B.sd_transformer_workspace_size(B.transformer_cfg(96, 96, 320))
     assert 0 < small < large
     assert B.status_string(5) == "workspace too small"
+
+
+def test_gemm_override_validation():
+    """The schedule hook accepts 0 or a multiple of 32 up to 256, and 0..16 splits."""
+    for bn, sp in [(48, 0), (512, 0), (-32, 0), (0, 17), (0, -1), (16, 1)]:
+        with pytest.raises(RuntimeError):
+            B.sd_gemm_override(bn, sp)
+    for bn, sp in [(32, 1), (256, 16), (160, 0), (0, 0)]:
+        B.sd_gemm_override(bn, sp)
