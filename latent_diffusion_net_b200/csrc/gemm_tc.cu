@@ -22,16 +22,32 @@ constexpr int kATileBytes = kBM * kBK * 2;  // 16 KB
 constexpr int kEpiThreads = 256;              // 8 epilogue warps, two per TMEM lane quarter
 constexpr int kGemmThreads = 64 + kEpiThreads;
 
+constexpr int kMaxStages = 12;
+constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA on sm_100
+constexpr int kSmemFixed = 1024 + 256 + 2048;  // alignment slack, barriers, per-column terms
+
 struct __align__(64) GemmMaps {
-  CUtensorMap a[kGemmMaxA];
+  CUtensorMap a[kGemmMaxA];   // BH x BW pixel boxes
+  CUtensorMap at[kGemmMaxA];  // (BH + 2) x BW boxes of the folded 3-tap segments
   CUtensorMap b[kGemmMaxB];
+};
+
+// A pipeline stage loads one 64-channel block of A and the matching B slices.
+// taps == 1: a BH x BW box shifted by (dx, dy) and one B slice at bk0.
+// taps == 3: the three vertically adjacent taps (dy = -1, 0, +1) of one column
+// dx of a 3x3 kernel share one (BH + 2) x BW box; tap t reads rows
+// [t*BW, t*BW + 128) of it (BW is a multiple of 8, so every view starts on a
+// 1024-byte swizzle atom) against the B slice at bk0 + t*bstep.
+struct KSeg {
+  int32_t amap, bmap, dx, dy, z, c0, bk0, nkb, taps, bstep;
 };
 
 struct GemmArgs {
   int32_t Ho, Wo, BH, BW, tiles_x, tiles_m, N;
-  int32_t nseg, total_kb;
+  int32_t nseg, total_kb;  // total_kb: pipeline stages of one output tile
   int32_t kb_per_split, splits, tiles_n, units;
-  GemmSeg seg[kGemmMaxSeg];
+  int32_t stages, stage_bytes, a_bytes;  // ring depth, bytes per stage, A region of a stage
+  KSeg seg[kGemmMaxSeg];
   GemmEpi epi;
   float* partial;  // split-K: FP32 [splits][Ho*Wo][N]; null otherwise
   int* err;
@@ -114,26 +130,27 @@ __device__ __forceinline__ void umma2_commit_both(uint64_t* bar) {
 // Roles (320 threads per CTA): warp 0 lane 0 TMA producer (both CTAs); warp 1
 // owns TMEM, lane 0 of the even CTA issues MMAs; warps 2-9 epilogue (TMEM lane
 // quarter warp % 4; warps 2-5 take the even 32-column chunks, 6-9 the odd ones).
-template <int BN, int STAGES>
+template <int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmArgs args) {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "epilogue works in 32-column chunks");
   constexpr int kBHalf = BN / 2;
   constexpr int kBTileBytes = kBHalf * kBK * 2;
-  constexpr int kStageBytes = kATileBytes + kBTileBytes;
   constexpr uint32_t kTmemCols = 512;  // two accumulators of up to 256 columns
   constexpr uint32_t kIdesc = umma_idesc_bf16(256, BN);
   constexpr int kChunks = BN / 32;
+  const int STAGES = args.stages;
+  const int stage_bytes = args.stage_bytes;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * stage_bytes);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* acc_full = empty_bar + STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;       // [2], used in the even CTA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* epi_col = reinterpret_cast<float*>(smem + STAGES * kStageBytes + 256);  // [2][256]
+  float* epi_col = reinterpret_cast<float*>(smem + STAGES * stage_bytes + 256);  // [2][256]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -164,10 +181,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int i = 0; i < kGemmMaxA; ++i) tma_prefetch_desc(&maps.a[i]);
+      for (int i = 0; i < kGemmMaxA; ++i) {
+        tma_prefetch_desc(&maps.a[i]);
+        tma_prefetch_desc(&maps.at[i]);
+      }
       tma_prefetch_desc(&maps.b[0]);
       tma_prefetch_desc(&maps.b[1]);
-      uint32_t q = 0;  // k-blocks issued by this CTA so far (stage ring position)
+      const uint32_t tall_bytes = (uint32_t)((args.BH + 2) * args.BW * kBK * 2 + 3 * kBTileBytes);
+      const uint32_t single_bytes = (uint32_t)(kATileBytes + kBTileBytes);
+      uint32_t q = 0;        // stages issued by this CTA so far
+      int s = 0;             // ring slot of stage q
+      uint32_t ph = 0;       // ring pass parity of stage q
       bool ok = true;
       for (int u = cluster_id; u < args.units && ok; u += nclusters) {
         const int z = u % args.splits;
@@ -179,58 +203,83 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int brow = nt * BN + (int)rank * kBHalf;
         const int kb_lo = z * args.kb_per_split;
         const int kb_hi = min(args.total_kb, kb_lo + args.kb_per_split);
-        int g = 0;
-        for (int si = 0; si < args.nseg && ok && g < kb_hi; ++si) {
-          const GemmSeg sg = args.seg[si];
-          for (int j = 0; j < sg.nkb; ++j, ++g) {
-            if (g < kb_lo) continue;
-            if (g >= kb_hi) break;
-            const uint32_t s = q % STAGES;
-            if (q >= (uint32_t)STAGES && !mbar_wait(&empty_bar[s], ((q / STAGES) - 1) & 1, abort_flag, args.err)) {
+        int g = 0;  // stage index of the first block of segment si
+        for (int si = 0; si < args.nseg && ok && g < kb_hi; g += args.seg[si].nkb, ++si) {
+          const KSeg sg = args.seg[si];
+          for (int j = max(0, kb_lo - g); j < sg.nkb && g + j < kb_hi; ++j) {
+            if (q >= (uint32_t)STAGES && !mbar_wait(&empty_bar[s], ph ^ 1, abort_flag, args.err)) {
               ok = false;
               break;
             }
-            uint8_t* a_dst = smem + s * kStageBytes;
-            uint8_t* b_dst = a_dst + kATileBytes;
-            if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * kStageBytes);
-            tma2_load_4d(a_dst, &maps.a[sg.amap], &full_bar[s], sg.c0 + j * kBK, tile_x0 + sg.dx, tile_y0 + sg.dy,
-                         sg.z);
-            tma2_load_2d(b_dst, &maps.b[sg.bmap], &full_bar[s], sg.bk0 + j * kBK, brow);
+            uint8_t* a_dst = smem + s * stage_bytes;
+            uint8_t* b_dst = a_dst + args.a_bytes;
+            const int kc = sg.c0 + j * kBK;
+            if (sg.taps == 3) {
+              if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * tall_bytes);
+              tma2_load_4d(a_dst, &maps.at[sg.amap], &full_bar[s], kc, tile_x0 + sg.dx, tile_y0 - 1, sg.z);
+#pragma unroll
+              for (int t = 0; t < 3; ++t)
+                tma2_load_2d(b_dst + t * kBTileBytes, &maps.b[sg.bmap], &full_bar[s], sg.bk0 + t * sg.bstep + j * kBK,
+                             brow);
+            } else {
+              if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * single_bytes);
+              tma2_load_4d(a_dst, &maps.a[sg.amap], &full_bar[s], kc, tile_x0 + sg.dx, tile_y0 + sg.dy, sg.z);
+              tma2_load_2d(b_dst, &maps.b[sg.bmap], &full_bar[s], sg.bk0 + j * kBK, brow);
+            }
             ++q;
+            if (++s == STAGES) {
+              s = 0;
+              ph ^= 1;
+            }
           }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      uint32_t q = 0;
+      const uint32_t view_bytes = (uint32_t)args.BW * kBK * 2;  // one pixel row of the tall box
+      int s = 0;
+      uint32_t ph = 0;
       int it = 0;
       bool ok = true;
       for (int u = cluster_id; u < args.units && ok; u += nclusters, ++it) {
         const int z = u % args.splits;
         const int kb_lo = z * args.kb_per_split;
-        const int nkb = min(args.total_kb, kb_lo + args.kb_per_split) - kb_lo;
+        const int kb_hi = min(args.total_kb, kb_lo + args.kb_per_split);
         const int b = it & 1;
         // the epilogues of both CTAs must have drained this accumulator (first use passes)
         if (!mbar_wait(&acc_empty[b], ((it >> 1) & 1) ^ 1, abort_flag, args.err)) break;
         tc_fence_after();
         const uint32_t tacc = tmem_base + (uint32_t)(b * 256);
-        for (int kb = 0; kb < nkb; ++kb, ++q) {
-          const uint32_t s = q % STAGES;
-          if (!mbar_wait(&full_bar[s], (q / STAGES) & 1, abort_flag, args.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
-          const uint64_t adesc = umma_desc_k_sw128(a_addr);
-          const uint64_t bdesc = umma_desc_k_sw128(a_addr + kATileBytes);
+        uint32_t acc = 0;  // the first MMA of a unit overwrites the accumulator
+        int g = 0;
+        for (int si = 0; si < args.nseg && ok && g < kb_hi; g += args.seg[si].nkb, ++si) {
+          const int taps = args.seg[si].taps;
+          const int nkb = args.seg[si].nkb;
+          for (int j = max(0, kb_lo - g); j < nkb && g + j < kb_hi; ++j) {
+            if (!mbar_wait(&full_bar[s], ph, abort_flag, args.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + s * stage_bytes);
+            const uint32_t b_addr = a_addr + (uint32_t)args.a_bytes;
+            for (int t = 0; t < taps; ++t) {
+              const uint64_t adesc = umma_desc_k_sw128(a_addr + (uint32_t)t * view_bytes);
+              const uint64_t bdesc = umma_desc_k_sw128(b_addr + (uint32_t)(t * kBTileBytes));
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            // +32 bytes along K inside the 128-byte swizzle row = +2 in the encoded address
-            umma2_bf16(tacc, adesc + 2 * k, bdesc + 2 * k, kIdesc, (kb | k) != 0 ? 1u : 0u);
+              for (int k = 0; k < kBK / 16; ++k) {
+                // +32 bytes along K inside the 128-byte swizzle row = +2 in the encoded address
+                umma2_bf16(tacc, adesc + 2 * k, bdesc + 2 * k, kIdesc, acc);
+                acc = 1;
+              }
+            }
+            umma2_commit_both(&empty_bar[s]);
+            if (++s == STAGES) {
+              s = 0;
+              ph ^= 1;
+            }
           }
-          umma2_commit_both(&empty_bar[s]);
         }
         if (ok) umma2_commit_both(&acc_full[b]);
       }
@@ -508,48 +557,15 @@ bool tmap_encode_4d(CUtensorMap* m, const void* ptr, const uint64_t d[4], uint32
 }
 
 template <int BN>
-struct Stages {
-  static constexpr int value = (kATileBytes + BN * kBK) * 8 <= 200 * 1024 ? 8 : 6;
-};
-
-template <int BN>
-static int launch_bn(const GemmMaps& maps, const GemmArgs& args, int grid, cudaStream_t st) {
-  constexpr int STAGES = Stages<BN>::value;
-  constexpr int kStageBytes = kATileBytes + (BN / 2) * kBK * 2;
-  constexpr size_t smem = 1024 + (size_t)STAGES * kStageBytes + 256 + 2048;
+static int launch_bn(const GemmMaps& maps, const GemmArgs& args, int grid, size_t smem, cudaStream_t st) {
   static bool attr_set = false;  // benign race: the attribute value is identical for every caller
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     if (e != cudaSuccess) return (int)e;
     attr_set = true;
   }
-  return (int)launch_pdl(gemm_tc_kernel<BN, STAGES>, dim3(grid), dim3(kGemmThreads), smem, st, maps, args);
+  return (int)launch_pdl(gemm_tc_kernel<BN>, dim3(grid), dim3(kGemmThreads), smem, st, maps, args);
 }
-
-static void choose_tile_rect(int Ho, int Wo, int* BH, int* BW) {
-  if (Ho == 1) {
-    *BH = 1;
-    *BW = 128;
-    return;
-  }
-  int best = -1, bw_best = 16;
-  const int cands[] = {16, 32, 8, 64, 4, 128};
-  for (int bw : cands) {
-    int bh = 128 / bw;
-    int tiles = ((Wo + bw - 1) / bw) * ((Ho + bh - 1) / bh);
-    if (best < 0 || tiles < best) {
-      best = tiles;
-      bw_best = bw;
-    }
-  }
-  *BW = bw_best;
-  *BH = 128 / bw_best;
-}
-
-struct GemmPlan {
-  int BH, BW, tiles_x, tiles_m, bn, tiles_n, splits, kb_per_split, total_kb, units, clusters;
-};
 
 static int sm_count() {
   static int num_sms = 0;
@@ -567,15 +583,13 @@ static int sm_count() {
 static int max_active_clusters() {
   static int n = 0;
   if (n == 0) {
-    constexpr int STAGES = Stages<256>::value;
-    constexpr size_t smem = 1024 + (size_t)STAGES * (kATileBytes + 128 * kBK * 2) + 256 + 2048;
-    cudaFuncSetAttribute(gemm_tc_kernel<256, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(gemm_tc_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (sm_count() / 2));
     cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = 200 * 1024;
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, gemm_tc_kernel<256, STAGES>, &cfg) != cudaSuccess || c <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&c, gemm_tc_kernel<256>, &cfg) != cudaSuccess || c <= 0) {
       cudaGetLastError();
       c = sm_count() / 2;
     }
@@ -584,29 +598,136 @@ static int max_active_clusters() {
   return n;
 }
 
-// Estimated cycles of a plan. Per k-block a CTA pair performs 2*256*BN*64 FLOPs
-// (2*BN cycles per SM at the tensor rate) and each SM loads 16 KB of A plus
-// BN*64 bytes of B (about 64 bytes per cycle per SM); the slower of the two
-// sets the pace. Units are spread over the clusters in rounds; the last
-// epilogue and the split-K reduction are added on top.
-static double plan_cost(int bn, int splits, int pairs, int N, int total_kb, long M, int clusters) {
+// Output tile rectangle of 128 pixels (BW x BH) with the fewest tiles. With
+// foldable 3x3 taps, narrow-and-tall rectangles come first: the shared box of
+// a tap column holds (BH + 2) rows for 3*BH rows of work.
+static void choose_tile_rect(int Ho, int Wo, bool prefer_tall, int* BH, int* BW) {
+  if (Ho == 1) {
+    *BH = 1;
+    *BW = 128;
+    return;
+  }
+  int best = -1, bw_best = 16;
+  const int plain[] = {16, 32, 8, 64, 4, 128};
+  const int tall[] = {8, 16, 32, 64, 4, 128};
+  for (int bw : prefer_tall ? tall : plain) {
+    const int bh = 128 / bw;
+    const int tiles = ((Wo + bw - 1) / bw) * ((Ho + bh - 1) / bh);
+    if (best < 0 || tiles < best) {
+      best = tiles;
+      bw_best = bw;
+    }
+  }
+  *BW = bw_best;
+  *BH = 128 / bw_best;
+}
+
+// Kernel segments of a problem: every group of three taps that differ only in
+// dy = -1, 0, +1 (same source, column, plane, channels and length, B offsets
+// bk0, bk0 + S, bk0 + 2S) becomes one 3-tap segment when `fold` is set.
+static int build_ksegs(const GemmProblem& p, bool fold, KSeg* out) {
+  bool used[kGemmMaxSeg] = {};
+  int n = 0;
+  for (int i = 0; i < p.nseg; ++i) {
+    if (used[i]) continue;
+    const GemmSeg& a = p.seg[i];
+    int mid = -1, hi = -1;
+    if (fold && a.dy == -1) {
+      for (int j = 0; j < p.nseg; ++j) {
+        const GemmSeg& c = p.seg[j];
+        if (used[j] || j == i || c.amap != a.amap || c.bmap != a.bmap || c.dx != a.dx || c.z != a.z ||
+            c.c0 != a.c0 || c.nkb != a.nkb)
+          continue;
+        if (c.dy == 0 && mid < 0) mid = j;
+      }
+      if (mid >= 0) {
+        const int S = p.seg[mid].bk0 - a.bk0;
+        for (int j = 0; j < p.nseg; ++j) {
+          const GemmSeg& c = p.seg[j];
+          if (used[j] || j == i || j == mid || c.amap != a.amap || c.bmap != a.bmap || c.dx != a.dx ||
+              c.z != a.z || c.c0 != a.c0 || c.nkb != a.nkb || c.dy != 1 || c.bk0 != a.bk0 + 2 * S)
+            continue;
+          hi = j;
+          break;
+        }
+      }
+    }
+    KSeg& k = out[n++];
+    k.amap = a.amap;
+    k.bmap = a.bmap;
+    k.dx = a.dx;
+    k.dy = a.dy;
+    k.z = a.z;
+    k.c0 = a.c0;
+    k.bk0 = a.bk0;
+    k.nkb = a.nkb;
+    k.taps = 1;
+    k.bstep = 0;
+    if (mid >= 0 && hi >= 0) {
+      k.taps = 3;
+      k.bstep = p.seg[mid].bk0 - a.bk0;
+      used[mid] = used[hi] = true;
+    }
+    used[i] = true;
+  }
+  return n;
+}
+
+struct GemmPlan {
+  int BH, BW, tiles_x, tiles_m, bn, tiles_n, splits, kb_per_split, total_kb, units, clusters;
+  int nkseg, stages, stage_bytes, a_bytes;
+  bool tall;
+  KSeg kseg[kGemmMaxSeg];
+};
+
+// Shared-memory layout of a stage for N tile bn.
+static void stage_layout(const GemmPlan& g, int bn, int* a_bytes, int* stage_bytes, int* stages) {
+  const int tall_a = (g.BH + 2) * g.BW * kBK * 2;
+  *a_bytes = g.tall ? std::max(kATileBytes, (tall_a + 1023) & ~1023) : kATileBytes;
+  *stage_bytes = *a_bytes + (g.tall ? 3 : 1) * (bn / 2) * kBK * 2;
+  *stages = std::min(kMaxStages, (kSmemLimit - kSmemFixed) / *stage_bytes);
+}
+
+// Estimated cycles of a plan. A CTA pair performs 2*256*BN*64 FLOPs per tap
+// and k-block (2*BN cycles per SM at the tensor rate); each SM takes its A box
+// and BN/2 rows of B per stage at about 50 bytes per cycle from L2, so a stage
+// costs the slower of the two. Units are spread over the clusters in rounds;
+// the split-K reduction is added on top.
+static double plan_cost(const GemmPlan& g, int bn, int splits, int pairs, int N, long M, int clusters) {
   const int tiles_n = (N + bn - 1) / bn;
   const long units = (long)pairs * tiles_n * splits;
   const long rounds = (units + clusters - 1) / clusters;
-  const int kb = (total_kb + splits - 1) / splits;
-  const double per_kb = std::max(2.0 * bn, 256.0 + bn);
-  double cost = (double)rounds * (kb * per_kb + 600.0) + 8.0 * bn;
+  double unit_cycles = 0;
+  const int a_tall = (g.BH + 2) * g.BW * kBK * 2;
+  for (int i = 0; i < g.nkseg; ++i) {
+    const KSeg& k = g.kseg[i];
+    const double mma = 2.0 * bn * k.taps;
+    const double load = ((k.taps == 3 ? a_tall : kATileBytes) + k.taps * (bn / 2) * kBK * 2.0) / 50.0;
+    unit_cycles += k.nkb * std::max(mma, load);
+  }
+  unit_cycles /= splits;
+  const double epilogue = 40.0 * bn;  // 8 warps drain 128 x BN FP32 values and store them
+  double cost = (double)rounds * (unit_cycles + 600.0) + epilogue;
+  if (rounds > 1) cost += (double)(rounds - 1) * std::max(0.0, epilogue - unit_cycles);
   if (splits > 1) cost += 4000.0 + (double)splits * M * N * 4.0 / 3000.0;
   return cost;
 }
 
 // Tile shape, N tile and split-K factor for a problem.
 static bool plan_gemm(const GemmProblem& p, GemmPlan* g) {
-  choose_tile_rect(p.Ho, p.Wo, &g->BH, &g->BW);
+  KSeg probe[kGemmMaxSeg];
+  bool foldable = false;
+  {
+    const int n = build_ksegs(p, true, probe);
+    for (int i = 0; i < n; ++i) foldable |= probe[i].taps == 3;
+  }
+  choose_tile_rect(p.Ho, p.Wo, foldable, &g->BH, &g->BW);
+  g->tall = foldable && g->BH >= 2 && g->BW % 8 == 0 && g->BW <= 16;
+  g->nkseg = build_ksegs(p, g->tall, g->kseg);
   g->tiles_x = (p.Wo + g->BW - 1) / g->BW;
   g->tiles_m = g->tiles_x * ((p.Ho + g->BH - 1) / g->BH);
   g->total_kb = 0;
-  for (int i = 0; i < p.nseg; ++i) g->total_kb += p.seg[i].nkb;
+  for (int i = 0; i < g->nkseg; ++i) g->total_kb += g->kseg[i].nkb;
   if (g->total_kb <= 0) return false;
   const int pairs = (g->tiles_m + 1) / 2;
   const int max_clusters = max_active_clusters();
@@ -627,11 +748,11 @@ static bool plan_gemm(const GemmProblem& p, GemmPlan* g) {
     for (int sp : sps) {
       if (p.force_splits) {
         if (sp != std::min(p.force_splits, g->total_kb)) continue;
-      } else if (sp > 1 && (g->total_kb / sp < 4 || (sp > 8 && sp % 2))) {
+      } else if (sp > 1 && (g->total_kb / sp < 2 || (sp > 8 && sp % 2))) {
         continue;
       }
       if (sp > 1 && (!p.splitk_ws || per_split * sp > p.splitk_ws_bytes || p.N % 8)) continue;
-      const double c = plan_cost(bn, sp, pairs, p.N, g->total_kb, M, max_clusters);
+      const double c = plan_cost(*g, bn, sp, pairs, p.N, M, max_clusters);
       if (best < 0 || c < best) {
         best = c;
         g->bn = bn;
@@ -645,7 +766,8 @@ static bool plan_gemm(const GemmProblem& p, GemmPlan* g) {
   g->splits = (g->total_kb + g->kb_per_split - 1) / g->kb_per_split;  // no empty split
   g->units = pairs * g->tiles_n * g->splits;
   g->clusters = std::min(g->units, max_clusters);
-  return true;
+  stage_layout(*g, g->bn, &g->a_bytes, &g->stage_bytes, &g->stages);
+  return g->stages >= 2;
 }
 
 int gemm_tc_plan_launches(const GemmProblem& p) {
@@ -667,13 +789,16 @@ int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   args.tiles_x = g.tiles_x;
   args.tiles_m = g.tiles_m;
   args.N = p.N;
-  args.nseg = p.nseg;
-  for (int i = 0; i < p.nseg; ++i) args.seg[i] = p.seg[i];
+  args.nseg = g.nkseg;
+  for (int i = 0; i < g.nkseg; ++i) args.seg[i] = g.kseg[i];
   args.total_kb = g.total_kb;
   args.kb_per_split = g.kb_per_split;
   args.splits = g.splits;
   args.tiles_n = g.tiles_n;
   args.units = g.units;
+  args.stages = g.stages;
+  args.stage_bytes = g.stage_bytes;
+  args.a_bytes = g.a_bytes;
   args.epi = p.epi;
   args.partial = g.splits > 1 ? p.splitk_ws : nullptr;
   args.err = p.err;
@@ -685,22 +810,28 @@ int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
     const GemmASrc& a = p.a[i < p.na ? i : 0];
     uint64_t d[4] = {(uint64_t)a.C, (uint64_t)a.W, (uint64_t)a.H, (uint64_t)a.Z};
     if (!tmap_encode_4d(&maps.a[i], a.ptr, d, args.BW, args.BH)) return -2;
+    if (g.tall) {
+      if (!tmap_encode_4d(&maps.at[i], a.ptr, d, args.BW, args.BH + 2)) return -2;
+    } else {
+      maps.at[i] = maps.a[i];
+    }
   }
   for (int i = 0; i < kGemmMaxB; ++i) {
     const GemmBSrc& b = p.b[i < p.nb ? i : 0];
     if (!tmap_encode_2d(&maps.b[i], b.ptr, (uint64_t)b.K, (uint64_t)b.rows, 64, (uint32_t)(bn / 2))) return -2;
   }
   const int grid = 2 * g.clusters;
+  const size_t smem = (size_t)kSmemFixed + (size_t)g.stages * g.stage_bytes;
   int e;
   switch (bn) {
-    case 32: e = launch_bn<32>(maps, args, grid, stream); break;
-    case 64: e = launch_bn<64>(maps, args, grid, stream); break;
-    case 96: e = launch_bn<96>(maps, args, grid, stream); break;
-    case 128: e = launch_bn<128>(maps, args, grid, stream); break;
-    case 160: e = launch_bn<160>(maps, args, grid, stream); break;
-    case 192: e = launch_bn<192>(maps, args, grid, stream); break;
-    case 224: e = launch_bn<224>(maps, args, grid, stream); break;
-    case 256: e = launch_bn<256>(maps, args, grid, stream); break;
+    case 32: e = launch_bn<32>(maps, args, grid, smem, stream); break;
+    case 64: e = launch_bn<64>(maps, args, grid, smem, stream); break;
+    case 96: e = launch_bn<96>(maps, args, grid, smem, stream); break;
+    case 128: e = launch_bn<128>(maps, args, grid, smem, stream); break;
+    case 160: e = launch_bn<160>(maps, args, grid, smem, stream); break;
+    case 192: e = launch_bn<192>(maps, args, grid, smem, stream); break;
+    case 224: e = launch_bn<224>(maps, args, grid, smem, stream); break;
+    case 256: e = launch_bn<256>(maps, args, grid, smem, stream); break;
     default: return -1;
   }
   if (e != 0 || g.splits <= 1) return e;
