@@ -32,15 +32,18 @@ struct __align__(64) GemmMaps {
   CUtensorMap b[kGemmMaxB];
 };
 
-// A pipeline stage loads one 64-channel block of A and the matching B slices.
-// taps == 1: a BH x BW box shifted by (dx, dy) and one B slice at bk0.
+// A pipeline stage carries at least 8 MMAs (the stage handshake costs about
+// as much as 4 of them):
+// taps == 1: `per` (1 or 2) consecutive 64-channel blocks, each a BH x BW box
+//   shifted by (dx, dy) against its B slice at bk0 + 64*j;
 // taps == 3: the three vertically adjacent taps (dy = -1, 0, +1) of one column
-// dx of a 3x3 kernel share one (BH + 2) x BW box; tap t reads rows
-// [t*BW, t*BW + 128) of it (BW is a multiple of 8, so every view starts on a
-// 1024-byte swizzle atom) against the B slice at bk0 + t*bstep.
+//   dx of a 3x3 kernel share one (BH + 2) x BW box of one channel block; tap t
+//   reads rows [t*BW, t*BW + 128) of it (BW is a multiple of 8, so every view
+//   starts on a 1024-byte swizzle atom) against the B slice at bk0 + t*bstep.
 struct KSeg {
-  int32_t amap, bmap, dx, dy, z, c0, bk0, nkb, taps, bstep;
+  int32_t amap, bmap, dx, dy, z, c0, bk0, nkb, taps, bstep, per;
 };
+__host__ __device__ inline int kseg_stages(const KSeg& k) { return (k.nkb + k.per - 1) / k.per; }
 
 struct GemmArgs {
   int32_t Ho, Wo, BH, BW, tiles_x, tiles_m, N;
@@ -203,28 +206,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int brow = nt * BN + (int)rank * kBHalf;
         const int kb_lo = z * args.kb_per_split;
         const int kb_hi = min(args.total_kb, kb_lo + args.kb_per_split);
-        int g = 0;  // stage index of the first block of segment si
-        for (int si = 0; si < args.nseg && ok && g < kb_hi; g += args.seg[si].nkb, ++si) {
+        int g = 0;  // index of the first stage of segment si
+        for (int si = 0; si < args.nseg && ok && g < kb_hi; g += kseg_stages(args.seg[si]), ++si) {
           const KSeg sg = args.seg[si];
-          for (int j = max(0, kb_lo - g); j < sg.nkb && g + j < kb_hi; ++j) {
+          const int nst = kseg_stages(sg);
+          for (int js = max(0, kb_lo - g); js < nst && g + js < kb_hi; ++js) {
             if (q >= (uint32_t)STAGES && !mbar_wait(&empty_bar[s], ph ^ 1, abort_flag, args.err)) {
               ok = false;
               break;
             }
             uint8_t* a_dst = smem + s * stage_bytes;
             uint8_t* b_dst = a_dst + args.a_bytes;
-            const int kc = sg.c0 + j * kBK;
+            const int j = js * sg.per;  // first channel block of this stage
             if (sg.taps == 3) {
               if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * tall_bytes);
-              tma2_load_4d(a_dst, &maps.at[sg.amap], &full_bar[s], kc, tile_x0 + sg.dx, tile_y0 - 1, sg.z);
+              tma2_load_4d(a_dst, &maps.at[sg.amap], &full_bar[s], sg.c0 + j * kBK, tile_x0 + sg.dx, tile_y0 - 1,
+                           sg.z);
 #pragma unroll
               for (int t = 0; t < 3; ++t)
                 tma2_load_2d(b_dst + t * kBTileBytes, &maps.b[sg.bmap], &full_bar[s], sg.bk0 + t * sg.bstep + j * kBK,
                              brow);
             } else {
-              if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * single_bytes);
-              tma2_load_4d(a_dst, &maps.a[sg.amap], &full_bar[s], kc, tile_x0 + sg.dx, tile_y0 + sg.dy, sg.z);
-              tma2_load_2d(b_dst, &maps.b[sg.bmap], &full_bar[s], sg.bk0 + j * kBK, brow);
+              const int nsub = min(sg.per, sg.nkb - j);
+              if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * nsub * single_bytes);
+              for (int h = 0; h < nsub; ++h) {
+                tma2_load_4d(a_dst + h * kATileBytes, &maps.a[sg.amap], &full_bar[s], sg.c0 + (j + h) * kBK,
+                             tile_x0 + sg.dx, tile_y0 + sg.dy, sg.z);
+                tma2_load_2d(b_dst + h * kBTileBytes, &maps.b[sg.bmap], &full_bar[s], sg.bk0 + (j + h) * kBK, brow);
+              }
             }
             ++q;
             if (++s == STAGES) {
@@ -253,10 +262,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const uint32_t tacc = tmem_base + (uint32_t)(b * 256);
         uint32_t acc = 0;  // the first MMA of a unit overwrites the accumulator
         int g = 0;
-        for (int si = 0; si < args.nseg && ok && g < kb_hi; g += args.seg[si].nkb, ++si) {
-          const int taps = args.seg[si].taps;
-          const int nkb = args.seg[si].nkb;
-          for (int j = max(0, kb_lo - g); j < nkb && g + j < kb_hi; ++j) {
+        for (int si = 0; si < args.nseg && ok && g < kb_hi; g += kseg_stages(args.seg[si]), ++si) {
+          const KSeg& sg = args.seg[si];
+          const int nst = kseg_stages(sg);
+          for (int js = max(0, kb_lo - g); js < nst && g + js < kb_hi; ++js) {
+            // operand pairs of this stage: three taps of one box, or up to `per` channel blocks
+            const int npair = sg.taps == 3 ? 3 : min(sg.per, sg.nkb - js * sg.per);
+            const uint32_t a_step = sg.taps == 3 ? view_bytes : (uint32_t)kATileBytes;
             if (!mbar_wait(&full_bar[s], ph, abort_flag, args.err)) {
               ok = false;
               break;
@@ -264,8 +276,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             tc_fence_after();
             const uint32_t a_addr = smem_u32(smem + s * stage_bytes);
             const uint32_t b_addr = a_addr + (uint32_t)args.a_bytes;
-            for (int t = 0; t < taps; ++t) {
-              const uint64_t adesc = umma_desc_k_sw128(a_addr + (uint32_t)t * view_bytes);
+            for (int t = 0; t < npair; ++t) {
+              const uint64_t adesc = umma_desc_k_sw128(a_addr + (uint32_t)t * a_step);
               const uint64_t bdesc = umma_desc_k_sw128(b_addr + (uint32_t)(t * kBTileBytes));
 #pragma unroll
               for (int k = 0; k < kBK / 16; ++k) {
@@ -663,9 +675,11 @@ static int build_ksegs(const GemmProblem& p, bool fold, KSeg* out) {
     k.nkb = a.nkb;
     k.taps = 1;
     k.bstep = 0;
+    k.per = a.nkb >= 2 ? 2 : 1;
     if (mid >= 0 && hi >= 0) {
       k.taps = 3;
       k.bstep = p.seg[mid].bk0 - a.bk0;
+      k.per = 1;
       used[mid] = used[hi] = true;
     }
     used[i] = true;
@@ -680,11 +694,24 @@ struct GemmPlan {
   KSeg kseg[kGemmMaxSeg];
 };
 
-// Shared-memory layout of a stage for N tile bn.
+// Shared-memory layout of a stage for N tile bn: the A region holds the
+// largest A operand of any segment (a tall box, or `per` boxes), the B region
+// the largest number of B slices.
 static void stage_layout(const GemmPlan& g, int bn, int* a_bytes, int* stage_bytes, int* stages) {
-  const int tall_a = (g.BH + 2) * g.BW * kBK * 2;
-  *a_bytes = g.tall ? std::max(kATileBytes, (tall_a + 1023) & ~1023) : kATileBytes;
-  *stage_bytes = *a_bytes + (g.tall ? 3 : 1) * (bn / 2) * kBK * 2;
+  const int tall_a = ((g.BH + 2) * g.BW * kBK * 2 + 1023) & ~1023;
+  int a = kATileBytes, nb = 1;
+  for (int i = 0; i < g.nkseg; ++i) {
+    const KSeg& k = g.kseg[i];
+    if (k.taps == 3) {
+      a = std::max(a, tall_a);
+      nb = std::max(nb, 3);
+    } else {
+      a = std::max(a, k.per * kATileBytes);
+      nb = std::max(nb, k.per);
+    }
+  }
+  *a_bytes = a;
+  *stage_bytes = a + nb * (bn / 2) * kBK * 2;
   *stages = std::min(kMaxStages, (kSmemLimit - kSmemFixed) / *stage_bytes);
 }
 
@@ -701,9 +728,12 @@ static double plan_cost(const GemmPlan& g, int bn, int splits, int pairs, int N,
   const int a_tall = (g.BH + 2) * g.BW * kBK * 2;
   for (int i = 0; i < g.nkseg; ++i) {
     const KSeg& k = g.kseg[i];
-    const double mma = 2.0 * bn * k.taps;
-    const double load = ((k.taps == 3 ? a_tall : kATileBytes) + k.taps * (bn / 2) * kBK * 2.0) / 50.0;
-    unit_cycles += k.nkb * std::max(mma, load);
+    // operand pairs per stage and the MMA cycles of one (a K=16 MMA takes at least ~54 cycles)
+    const int pairs_per_stage = k.taps == 3 ? 3 : k.per;
+    const double mma = pairs_per_stage * 4.0 * std::max(54.0, bn / 2.0);
+    const double load =
+        ((k.taps == 3 ? a_tall : k.per * kATileBytes) + pairs_per_stage * (bn / 2) * kBK * 2.0) / 50.0;
+    unit_cycles += kseg_stages(k) * std::max(std::max(mma, load), 520.0);  // 520: stage handshake
   }
   unit_cycles /= splits;
   const double epilogue = 40.0 * bn;  // 8 warps drain 128 x BN FP32 values and store them
@@ -724,10 +754,18 @@ static bool plan_gemm(const GemmProblem& p, GemmPlan* g) {
   choose_tile_rect(p.Ho, p.Wo, foldable, &g->BH, &g->BW);
   g->tall = foldable && g->BH >= 2 && g->BW % 8 == 0 && g->BW <= 16;
   g->nkseg = build_ksegs(p, g->tall, g->kseg);
+  bool any_tall = false;
+  for (int i = 0; i < g->nkseg; ++i) any_tall |= g->kseg[i].taps == 3;
+  if (any_tall) {
+    // the few single blocks beside tall stages (a fused 1x1 shortcut) keep one
+    // block per stage so the stage stays at the tall size
+    for (int i = 0; i < g->nkseg; ++i)
+      if (g->kseg[i].taps == 1) g->kseg[i].per = 1;
+  }
   g->tiles_x = (p.Wo + g->BW - 1) / g->BW;
   g->tiles_m = g->tiles_x * ((p.Ho + g->BH - 1) / g->BH);
   g->total_kb = 0;
-  for (int i = 0; i < g->nkseg; ++i) g->total_kb += g->kseg[i].nkb;
+  for (int i = 0; i < g->nkseg; ++i) g->total_kb += kseg_stages(g->kseg[i]);
   if (g->total_kb <= 0) return false;
   const int pairs = (g->tiles_m + 1) / 2;
   const int max_clusters = max_active_clusters();
