@@ -57,6 +57,7 @@ constexpr int kMaxGroups = 64;
 constexpr size_t kGnAccBytes = (size_t)kMaxGnLaunches * 2 * kMaxGroups * sizeof(unsigned long long);
 constexpr int kMaxStatBlocks = 512;  // GroupNorm partial-sum slots: 2 CTAs per SM, up to 256 SMs
 
+
 struct Arena {
   uint8_t* base;
   size_t off;
@@ -77,6 +78,8 @@ struct Ctx {
   int* gn_seq;                 // host: GroupNorm launches issued so far in this call
   float* skws;  // split-K FP32 partial products
   size_t skws_bytes;
+  float* attn_part;   // pieces of split attention items
+  size_t attn_part_bytes;
   int sms;
 };
 
@@ -93,6 +96,8 @@ Ctx make_ctx(Arena& ar, cudaStream_t st, int sms) {
   c.skws_bytes = kSplitKBytes;
   c.st = st;
   c.sms = sms < kMaxStatBlocks / 2 ? sms : kMaxStatBlocks / 2;
+  c.attn_part_bytes = sdk::attention_partial_bytes(kMaxStatBlocks / 2);
+  c.attn_part = static_cast<float*>(ar.take(c.attn_part_bytes));
   return c;
 }
 
@@ -315,9 +320,10 @@ int run_ln(const Ctx& c, const bf16* x, int N, int C, const bf16* g, const bf16*
 int run_attn(const Ctx& c, const bf16* qbase, int q_ld, int q_col, const bf16* kvbase, int kv_ld, int k_col,
              int v_col, bf16* o, int ldo, int Nq, int Nk, int heads) {
   const double C = 64.0 * heads;
-  sdp::Scope sc("attention", sdp::F_ATTN, 4.0 * Nq * Nk * C, 2.0 * C * (2.0 * Nq + 2.0 * Nk), c.st);
+  sdp::Scope sc("attention", sdp::F_ATTN, 4.0 * Nq * Nk * C, 2.0 * C * (2.0 * Nq + 2.0 * Nk), c.st,
+                sdk::attention_plan_launches(Nq, Nk, heads, c.sms));
   return sdk::launch_attention_tc(qbase, q_ld, Nq, q_col, kvbase, kv_ld, Nk, k_col, v_col, o, ldo, Nq, Nk, heads,
-                                  c.err, c.st);
+                                  c.attn_part, c.attn_part_bytes, c.sms, c.err, c.st);
 }
 
 // Transformer2DModel; y may alias x.

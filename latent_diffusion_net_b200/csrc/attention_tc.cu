@@ -5,7 +5,16 @@
 // self-attention over the H*W image tokens (Q = K = V source) and for
 // cross-attention over the 77 context rows.
 //
-// One CTA = 128 queries of one head; 192 threads:
+// Work: every (head, 128-query tile) item runs over ceil(Nk/128) key tiles.
+// The grid is persistent (two CTAs per SM) and the sequence of all
+// (item, key tile) steps is cut into equal contiguous ranges, one per CTA, so
+// no SM idles while another finishes a second wave. An item whose key tiles
+// are split between CTAs leaves one piece per CTA in a workspace slot (its
+// unnormalised output with its running maximum and row sum); a small merge
+// kernel then combines the pieces of each split item in CTA order. Splitting is
+// used only where it shortens the longest CTA.
+//
+// 192 threads per CTA:
 //   warps 0-3  softmax: thread i owns query row i (TMEM lane i). Per 128-key
 //              tile it reads its S row from TMEM, keeps a running maximum in the
 //              log2 domain, writes P = exp2(s*log2e/8 - m) as BF16 into shared
@@ -13,7 +22,7 @@
 //              accumulates the row sum in a register. The output O lives in TMEM
 //              and is rescaled only when the running maximum grew by more than
 //              2^8 since the last rescale (P values stay <= 256, exact in FP32).
-//   warp 4     TMA producer: Q once, then K tiles (double-buffered) and V
+//   warp 4     TMA producer: Q once per item, K tiles (double-buffered) and V
 //              tiles (single buffer, reloaded once the previous PV product is
 //              done), zero-filled past the last key.
 //   warp 5     MMA issuer (one thread): S = Q K^T (M=128, N=128, K=64) and
@@ -24,6 +33,7 @@
 #include "common.cuh"
 #include "kernels.cuh"
 
+#include <algorithm>
 #include <mutex>
 
 #include "gemm_tc.cuh"
@@ -102,8 +112,18 @@ struct AttnArgs {
   __nv_bfloat16* O;
   int32_t ldo;
   float scale_log2;
+  int32_t qtiles, ktiles;  // 128-query tiles per head, 128-key tiles per item
+  int64_t steps;           // heads * qtiles * ktiles
+  int32_t ctas;            // grid size: CTA c runs steps [c*steps/ctas, (c+1)*steps/ctas)
+  float* partial;          // [ctas][2] slots of kSlotFloats (pieces of split items)
   int* err;
 };
+
+constexpr int kSlotFloats = 128 * 64 + 2 * 128;  // O rows, then running maxima, then row sums
+
+__host__ __device__ inline int64_t cta_first_step(int64_t c, int64_t steps, int64_t ctas) {
+  return c * steps / ctas;
+}
 
 }  // namespace
 
@@ -125,14 +145,15 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* p_full = bars + 8;
   uint64_t* pv_done = bars + 9;
   uint64_t* s_free = bars + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* q_empty = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * kAQ;
-  const int h = blockIdx.y;
-  const int ntiles = (args.Nk + kAK - 1) / kAK;
+  const int nt = args.ktiles;
+  const int w0 = (int)cta_first_step(blockIdx.x, args.steps, args.ctas);  // first step of this CTA
+  const int T = (int)cta_first_step(blockIdx.x + 1, args.steps, args.ctas) - w0;  // steps of this CTA
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -146,6 +167,7 @@ __global__ void __launch_bounds__(192, 2)
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
     mbar_init(s_free, 128);
+    mbar_init(q_empty, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -164,14 +186,22 @@ __global__ void __launch_bounds__(192, 2)
     if (lane == 0) {
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.kv);
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      tma_load_2d(sQ, &maps.q, q_full, args.q_col + h * 64, q0);
-      for (int j = 0; j < ntiles; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&k_empty[s], ((j >> 1) - 1) & 1, abort_flag, args.err)) break;
+      int ii = 0;  // items started
+      int X = (int)(w0 / nt), j = (int)(w0 % nt);
+      for (int t = 0; t < T; ++t, j = (j + 1 == nt) ? 0 : j + 1, X += (j == 0)) {
+        const int h = X / args.qtiles, qt = X % args.qtiles;
+        if (t == 0 || j == 0) {
+          // Q of a new item once every S product of the previous one is done
+          if (ii > 0 && !mbar_wait(q_empty, (ii - 1) & 1, abort_flag, args.err)) break;
+          mbar_arrive_expect_tx(q_full, kTileBytes);
+          tma_load_2d(sQ, &maps.q, q_full, args.q_col + h * 64, qt * kAQ);
+          ++ii;
+        }
+        const int s = t & 1;
+        if (t >= 2 && !mbar_wait(&k_empty[s], ((t >> 1) - 1) & 1, abort_flag, args.err)) break;
         mbar_arrive_expect_tx(&k_full[s], kTileBytes);
         tma_load_2d(sK + s * kTileBytes, &maps.kv, &k_full[s], args.k_col + h * 64, j * kAK);
-        if (j >= 1 && !mbar_wait(v_empty, (j - 1) & 1, abort_flag, args.err)) break;
+        if (t >= 1 && !mbar_wait(v_empty, (t - 1) & 1, abort_flag, args.err)) break;
         mbar_arrive_expect_tx(v_full, kTileBytes);
         tma_load_2d(sV, &maps.kv, v_full, args.v_col + h * 64, j * kAK);
       }
@@ -181,45 +211,48 @@ __global__ void __launch_bounds__(192, 2)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_attn(128, false);
       constexpr uint32_t kIdO = idesc_attn(64, true);
-      bool ok = mbar_wait(q_full, 0, abort_flag, args.err);
       const uint64_t qdesc = umma_desc_k_sw128(smem_u32(sQ));
-      // S_0
-      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, args.err);
-      if (ok) {
-        tc_fence_after();
-        const uint64_t kdesc = umma_desc_k_sw128(smem_u32(sK));
-#pragma unroll
-        for (int k = 0; k < 4; ++k) umma_bf16(tS, qdesc + 2 * k, kdesc + 2 * k, kIdS, k > 0 ? 1u : 0u);
-        umma_commit(&k_empty[0]);
-        umma_commit(s_full);
-      }
-      for (int j = 0; j < ntiles && ok; ++j) {
-        // S_{j+1} as soon as the softmax warps hold S_j in registers
-        if (j + 1 < ntiles) {
-          const int s1 = (j + 1) & 1;
-          if (!mbar_wait(s_free, j & 1, abort_flag, args.err)) break;
-          if (!mbar_wait(&k_full[s1], ((j + 1) >> 1) & 1, abort_flag, args.err)) break;
+      int ii = 0;                // items whose Q has been waited for
+      int jS = (int)(w0 % nt);   // key tile of S_t
+      int jP = jS;               // key tile of the PV product of step t - 1
+      // step t issues S_t (once the softmax warps hold S_{t-1} in registers), then
+      // O += P_{t-1} V_{t-1}
+      for (int t = 0; t <= T; ++t) {
+        if (t < T) {
+          if (t > 0 && !mbar_wait(s_free, (t - 1) & 1, abort_flag, args.err)) break;
+          if (t == 0 || jS == 0) {
+            if (!mbar_wait(q_full, ii & 1, abort_flag, args.err)) break;
+            ++ii;
+          }
+          const int s = t & 1;
+          if (!mbar_wait(&k_full[s], (t >> 1) & 1, abort_flag, args.err)) break;
           tc_fence_after();
-          const uint64_t kdesc = umma_desc_k_sw128(smem_u32(sK + s1 * kTileBytes));
+          const uint64_t kdesc = umma_desc_k_sw128(smem_u32(sK + s * kTileBytes));
 #pragma unroll
           for (int k = 0; k < 4; ++k) umma_bf16(tS, qdesc + 2 * k, kdesc + 2 * k, kIdS, k > 0 ? 1u : 0u);
-          umma_commit(&k_empty[s1]);
+          umma_commit(&k_empty[s]);
           umma_commit(s_full);
+          if (t == T - 1 || jS == nt - 1) umma_commit(q_empty);  // last S of this item
+          jS = (jS + 1 == nt) ? 0 : jS + 1;
         }
-        // O += P_j V_j once the softmax of tile j has written P_j and V_j has landed
-        if (!mbar_wait(p_full, j & 1, abort_flag, args.err)) break;
-        if (!mbar_wait(v_full, j & 1, abort_flag, args.err)) break;
-        tc_fence_after();
-        const uint32_t vbase = smem_u32(sV);
+        if (t > 0) {
+          const int tp = t - 1;
+          if (!mbar_wait(p_full, tp & 1, abort_flag, args.err)) break;
+          if (!mbar_wait(v_full, tp & 1, abort_flag, args.err)) break;
+          tc_fence_after();
+          const bool first = tp == 0 || jP == 0;
+          const uint32_t vbase = smem_u32(sV);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          // keys [16k, 16k + 16): P half k/4 at +32 bytes per step; V rows 16k.. (+2048 bytes per step)
-          const uint64_t pdesc = umma_desc_k_sw128(smem_u32(sP + (k >> 2) * kTileBytes)) + 2 * (k & 3);
-          const uint64_t vdesc = umma_desc_mn_sw128(vbase + k * 2048);
-          umma_bf16(tO, pdesc, vdesc, kIdO, (j > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 8; ++k) {
+            // keys [16k, 16k + 16): P half k/4 at +32 bytes per step; V rows 16k.. (+2048 bytes per step)
+            const uint64_t pdesc = umma_desc_k_sw128(smem_u32(sP + (k >> 2) * kTileBytes)) + 2 * (k & 3);
+            const uint64_t vdesc = umma_desc_mn_sw128(vbase + k * 2048);
+            umma_bf16(tO, pdesc, vdesc, kIdO, (!first || k > 0) ? 1u : 0u);
+          }
+          umma_commit(v_empty);
+          umma_commit(pv_done);
+          jP = (jP + 1 == nt) ? 0 : jP + 1;
         }
-        umma_commit(v_empty);
-        umma_commit(pv_done);
       }
     }
   } else {
@@ -229,16 +262,17 @@ __global__ void __launch_bounds__(192, 2)
     const float sl2 = args.scale_log2;
     float m_used = -INFINITY;  // maximum the stored P and O are relative to (log2 domain)
     float l = 0.f;
-    bool ok = true;
+    bool whole = true;  // this CTA holds the item from its first key tile
     uint8_t* prow0 = sP + row * 128;
-    for (int j = 0; j < ntiles; ++j) {
-      if (!mbar_wait(s_full, j & 1, abort_flag, args.err)) {
-        ok = false;
-        break;
-      }
+    int X = (int)(w0 / nt), j = (int)(w0 % nt);
+    for (int t = 0; t < T; ++t, j = (j + 1 == nt) ? 0 : j + 1, X += (j == 0)) {
+      const bool first = t == 0 || j == 0;
+      const bool last = t == T - 1 || j == nt - 1;
+      if (first) whole = j == 0;
+      if (!mbar_wait(s_full, t & 1, abort_flag, args.err)) break;
       tc_fence_after();
       const int kvalid = args.Nk - j * kAK;  // keys of this tile that exist
-      // the whole S row into registers, then hand the TMEM columns back for S_{j+1}
+      // the whole S row into registers, then hand the TMEM columns back for S_{t+1}
       uint32_t sv[128];
       tmem_ld_32x32b_x32(tS + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_ld_32x32b_x32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
@@ -258,29 +292,29 @@ __global__ void __launch_bounds__(192, 2)
           mx = fmaxf(mx, __uint_as_float(sv[i]));
         }
       }
-      const float m_new = fmaxf(m_used, mx * sl2);
       // the previous PV product must be done before P is overwritten or O rescaled
-      if (j > 0 && !mbar_wait(pv_done, (j - 1) & 1, abort_flag, args.err)) {
-        ok = false;
-        break;
-      }
+      if (t > 0 && !mbar_wait(pv_done, (t - 1) & 1, abort_flag, args.err)) break;
       tc_fence_after();
-      if (j == 0) {
-        m_used = m_new;
-      } else if (m_new > m_used + 8.f) {
-        const float alpha = ex2(m_used - m_new);
-        l *= alpha;
+      if (first) {
+        m_used = mx * sl2;
+        l = 0.f;
+      } else {
+        const float m_new = fmaxf(m_used, mx * sl2);
+        if (m_new > m_used + 8.f) {
+          const float alpha = ex2(m_used - m_new);
+          l *= alpha;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tO + lane_off + c * 32, r);
-          tmem_ld_wait();
+          for (int c = 0; c < 2; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tO + lane_off + c * 32, r);
+            tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st_32x32b_x32(tO + lane_off + c * 32, r);
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st_32x32b_x32(tO + lane_off + c * 32, r);
+          }
+          tmem_st_wait();
+          m_used = m_new;
         }
-        tmem_st_wait();
-        m_used = m_new;
       }
       // P = exp2(s*scale*log2e - m_used) in BF16 (masked keys give exp2(-inf) = 0), row sum
 #pragma unroll
@@ -304,29 +338,52 @@ __global__ void __launch_bounds__(192, 2)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
-    }
-    // epilogue: O / l
-    if (ok && mbar_wait(pv_done, (ntiles - 1) & 1, abort_flag, args.err)) {
+      if (!last) continue;
+
+      // ---------------------------------------------------------- end of this CTA's part of item X
+      if (!mbar_wait(pv_done, t & 1, abort_flag, args.err)) break;
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int qrow = q0 + row;
+      const int h = X / args.qtiles;
+      const int qrow = (X % args.qtiles) * kAQ + row;
       __nv_bfloat16* dst = args.O + (size_t)qrow * args.ldo + h * 64;
+      if (whole && j == nt - 1) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tO + lane_off + c * 32, r);
+          tmem_ld_wait();
+          if (qrow < args.Nq) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              d4[u] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * u]) * inv, __uint_as_float(r[8 * u + 1]) * inv),
+                                 pack_bf16x2(__uint_as_float(r[8 * u + 2]) * inv, __uint_as_float(r[8 * u + 3]) * inv),
+                                 pack_bf16x2(__uint_as_float(r[8 * u + 4]) * inv, __uint_as_float(r[8 * u + 5]) * inv),
+                                 pack_bf16x2(__uint_as_float(r[8 * u + 6]) * inv, __uint_as_float(r[8 * u + 7]) * inv));
+            }
+          }
+        }
+        tc_fence_before();
+        continue;
+      }
+      // a piece of a split item: leave it in this CTA's slot (0 for its first item, 1 otherwise)
+      // for the merge kernel that runs after this one
+      float* slot = args.partial + ((size_t)blockIdx.x * 2 + (X == (int)(w0 / nt) ? 0 : 1)) * kSlotFloats;
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tO + lane_off + c * 32, r);
         tmem_ld_wait();
-        if (qrow < args.Nq) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+        float4* o4 = reinterpret_cast<float4*>(slot + row * 64 + c * 32);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            d4[u] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * u]) * inv, __uint_as_float(r[8 * u + 1]) * inv),
-                               pack_bf16x2(__uint_as_float(r[8 * u + 2]) * inv, __uint_as_float(r[8 * u + 3]) * inv),
-                               pack_bf16x2(__uint_as_float(r[8 * u + 4]) * inv, __uint_as_float(r[8 * u + 5]) * inv),
-                               pack_bf16x2(__uint_as_float(r[8 * u + 6]) * inv, __uint_as_float(r[8 * u + 7]) * inv));
-          }
-        }
+        for (int u = 0; u < 8; ++u)
+          __stcg(o4 + u, make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                                     __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3])));
       }
+      tc_fence_before();
+      __stcg(slot + 8192 + row, m_used);
+      __stcg(slot + 8320 + row, l);
     }
   }
 
@@ -336,9 +393,87 @@ __global__ void __launch_bounds__(192, 2)
   if (warp == 5) tmem_dealloc(tmem, kTmemCols);
 }
 
+// Merge of split items: block b looks at the boundary between CTAs b and b+1;
+// if it falls inside an item and is that item's first boundary, the block
+// merges the item's pieces in CTA order: M = max m_p, O = sum 2^(m_p - M) O_p /
+// sum 2^(m_p - M) l_p. Two threads per query row, 32 output columns each.
+__global__ void __launch_bounds__(256) attention_merge_kernel(const __grid_constant__ AttnArgs args) {
+  pdl_wait();
+  pdl_trigger();
+  const int nt = args.ktiles;
+  const int64_t b = blockIdx.x + 1;
+  const int64_t s0 = cta_first_step(b, args.steps, args.ctas);
+  if (s0 % nt == 0) return;                                            // boundary between items
+  if (cta_first_step(b - 1, args.steps, args.ctas) / nt == s0 / nt &&
+      cta_first_step(b - 1, args.steps, args.ctas) % nt != 0)
+    return;                                                            // an earlier boundary merges it
+  const int X = (int)(s0 / nt);
+  const int64_t s_lo = (int64_t)X * nt, s_hi = s_lo + nt - 1;
+  int64_t c_lo = b - 1, c_hi = b;
+  while (c_hi + 1 < args.ctas && cta_first_step(c_hi + 1, args.steps, args.ctas) <= s_hi) ++c_hi;
+  (void)s_lo;
+  const int row = threadIdx.x >> 1, half = threadIdx.x & 1;
+  float mmax = -INFINITY;
+  for (int64_t c = c_lo; c <= c_hi; ++c) {
+    const int fi = (int)(cta_first_step(c, args.steps, args.ctas) / nt);
+    const float* sl = args.partial + ((size_t)c * 2 + (X == fi ? 0 : 1)) * kSlotFloats;
+    mmax = fmaxf(mmax, __ldcg(sl + 8192 + row));
+  }
+  float acc[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+  float lsum = 0.f;
+  for (int64_t c = c_lo; c <= c_hi; ++c) {
+    const int fi = (int)(cta_first_step(c, args.steps, args.ctas) / nt);
+    const float* sl = args.partial + ((size_t)c * 2 + (X == fi ? 0 : 1)) * kSlotFloats;
+    const float e = ex2(__ldcg(sl + 8192 + row) - mmax);
+    lsum += e * __ldcg(sl + 8320 + row);
+    const float4* o4 = reinterpret_cast<const float4*>(sl + row * 64 + half * 32);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float4 v = __ldcg(o4 + u);
+      acc[4 * u] += e * v.x;
+      acc[4 * u + 1] += e * v.y;
+      acc[4 * u + 2] += e * v.z;
+      acc[4 * u + 3] += e * v.w;
+    }
+  }
+  const int h = X / args.qtiles;
+  const int qrow = (X % args.qtiles) * kAQ + row;
+  if (qrow >= args.Nq) return;
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+  uint4* d4 = reinterpret_cast<uint4*>(args.O + (size_t)qrow * args.ldo + h * 64 + half * 32);
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    d4[u] = make_uint4(pack_bf16x2(acc[8 * u] * inv, acc[8 * u + 1] * inv),
+                       pack_bf16x2(acc[8 * u + 2] * inv, acc[8 * u + 3] * inv),
+                       pack_bf16x2(acc[8 * u + 4] * inv, acc[8 * u + 5] * inv),
+                       pack_bf16x2(acc[8 * u + 6] * inv, acc[8 * u + 7] * inv));
+}
+
+size_t attention_partial_bytes(int num_sms) { return (size_t)2 * num_sms * 2 * kSlotFloats * sizeof(float); }
+
+// Split the key tiles of items between CTAs only when that shortens the
+// longest CTA: with whole items a CTA alone on its SM runs a step in about 0.6
+// of the time two co-resident CTAs take; a split adds about two steps of
+// overhead (the pieces and their merge).
+static bool attention_split_pays(int items, int ktiles, int num_sms) {
+  if (ktiles < 2) return false;
+  const int resident = 2 * num_sms;
+  const double whole = items <= num_sms ? 0.6 * ktiles : (double)((items + resident - 1) / resident) * ktiles;
+  const double split = (double)items * ktiles / resident + 2.0;
+  return split < whole;
+}
+
+int attention_plan_launches(int Nq, int Nk, int heads, int num_sms) {
+  const int items = heads * ((Nq + kAQ - 1) / kAQ);
+  return attention_split_pays(items, (Nk + kAK - 1) / kAK, num_sms) ? 2 : 1;
+}
+
 int launch_attention_tc(const __nv_bfloat16* qbase, int q_ld, int q_rows, int q_col, const __nv_bfloat16* kvbase,
                         int kv_ld, int kv_rows, int k_col, int v_col, __nv_bfloat16* O, int ldo, int Nq, int Nk,
-                        int heads, int* err, cudaStream_t st) {
+                        int heads, float* partial, size_t partial_bytes, int num_sms, int* err, cudaStream_t st) {
+  if (Nq <= 0 || Nk <= 0 || heads <= 0) return 0;
   AttnMaps maps;
   memset(&maps, 0, sizeof(maps));
   if (!tmap_encode_2d(&maps.q, qbase, (uint64_t)q_ld, (uint64_t)q_rows, 64, 128)) return -2;
@@ -352,6 +487,16 @@ int launch_attention_tc(const __nv_bfloat16* qbase, int q_ld, int q_rows, int q_
   a.O = O;
   a.ldo = ldo;
   a.scale_log2 = 0.125f * 1.4426950408889634f;
+  a.qtiles = (Nq + kAQ - 1) / kAQ;
+  a.ktiles = (Nk + kAK - 1) / kAK;
+  const int items = heads * a.qtiles;
+  a.steps = (int64_t)items * a.ktiles;
+  const int resident = 2 * num_sms;
+  const bool split = partial && partial_bytes >= attention_partial_bytes(num_sms) &&
+                     attention_split_pays(items, a.ktiles, num_sms);
+  // split: every CTA an equal share of the steps; otherwise one CTA per whole item
+  a.ctas = split ? (int)std::min<int64_t>(resident, a.steps) : items;
+  a.partial = partial;
   a.err = err;
   constexpr size_t smem = 1024 + 6 * kTileBytes + 128;
   static bool attr = false;  // benign race: identical value for every caller
@@ -360,8 +505,9 @@ int launch_attention_tc(const __nv_bfloat16* qbase, int q_ld, int q_rows, int q_
     if (e != cudaSuccess) return (int)e;
     attr = true;
   }
-  dim3 grid((Nq + kAQ - 1) / kAQ, heads);
-  return (int)launch_pdl(attention_tc_kernel, grid, dim3(192), smem, st, maps, a);
+  int e = (int)launch_pdl(attention_tc_kernel, dim3(a.ctas), dim3(192), smem, st, maps, a);
+  if (e != 0 || !split || a.ctas < 2) return e;
+  return (int)launch_pdl(attention_merge_kernel, dim3(a.ctas - 1), dim3(256), 0, st, a);
 }
 
 }  // namespace sdk

@@ -50,10 +50,16 @@ int launch_conv_in_im2col(const __nv_bfloat16* s0, int c0, const __nv_bfloat16* 
 
 // Flash attention on tcgen05 (head_dim 64): O[i, h*64 + d] = softmax_j(Q_i.K_j / 8) V_j
 // per head; Q rows come from a [q_rows, q_ld] matrix at column q_col + 64h, K and V
-// from a [kv_rows, kv_ld] matrix at columns k_col + 64h and v_col + 64h.
+// from a [kv_rows, kv_ld] matrix at columns k_col + 64h and v_col + 64h. Where it
+// pays, the key tiles of the (head, query tile) items are spread evenly over
+// 2*num_sms CTAs; the pieces of split items go through `partial`
+// (attention_partial_bytes(num_sms) bytes; null disables splitting) and are merged
+// by a second kernel. attention_plan_launches gives the number of kernels (1 or 2).
+size_t attention_partial_bytes(int num_sms);
+int attention_plan_launches(int Nq, int Nk, int heads, int num_sms);
 int launch_attention_tc(const __nv_bfloat16* qbase, int q_ld, int q_rows, int q_col, const __nv_bfloat16* kvbase,
                         int kv_ld, int kv_rows, int k_col, int v_col, __nv_bfloat16* O, int ldo, int Nq, int Nk,
-                        int heads, int* err, cudaStream_t st);
+                        int heads, float* partial, size_t partial_bytes, int num_sms, int* err, cudaStream_t st);
 
 // Flash attention (head_dim 64) on mma.sync: O[i, h*64 + d] = softmax_j(Q_i.K_j / 8) V_j per head.
 int launch_attention(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk, const __nv_bfloat16* V,
