@@ -127,6 +127,52 @@ __host__ __device__ inline int64_t cta_first_step(int64_t c, int64_t steps, int6
 
 }  // namespace
 
+// End of a CTA's part of item X (one query row per thread, O in TMEM at
+// tOrow): a whole item is normalised and stored as BF16; a piece of a split
+// item goes to this CTA's workspace slot (0 for its first item, 1 otherwise)
+// for the merge kernel. Kept out of line: it runs once per item and its
+// registers would otherwise compete with the S row of the softmax loop.
+__device__ __noinline__ void attn_item_end(const AttnArgs& args, uint32_t tOrow, int row, int X, bool whole,
+                                           bool first_item, float m_used, float l) {
+  const int h = X / args.qtiles;
+  const int qrow = (X % args.qtiles) * kAQ + row;
+  if (whole) {
+    __nv_bfloat16* dst = args.O + (size_t)qrow * args.ldo + h * 64;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tOrow + c * 32, r);
+      tmem_ld_wait();
+      if (qrow < args.Nq) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          d4[u] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * u]) * inv, __uint_as_float(r[8 * u + 1]) * inv),
+                             pack_bf16x2(__uint_as_float(r[8 * u + 2]) * inv, __uint_as_float(r[8 * u + 3]) * inv),
+                             pack_bf16x2(__uint_as_float(r[8 * u + 4]) * inv, __uint_as_float(r[8 * u + 5]) * inv),
+                             pack_bf16x2(__uint_as_float(r[8 * u + 6]) * inv, __uint_as_float(r[8 * u + 7]) * inv));
+        }
+      }
+    }
+    return;
+  }
+  float* slot = args.partial + ((size_t)blockIdx.x * 2 + (first_item ? 0 : 1)) * kSlotFloats;
+#pragma unroll 1
+  for (int c = 0; c < 2; ++c) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tOrow + c * 32, r);
+    tmem_ld_wait();
+    float4* o4 = reinterpret_cast<float4*>(slot + row * 64 + c * 32);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      __stcg(o4 + u, make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
+                                 __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3])));
+  }
+  __stcg(slot + 8192 + row, m_used);
+  __stcg(slot + 8320 + row, l);
+}
+
 __global__ void __launch_bounds__(192, 2)
     attention_tc_kernel(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -258,26 +304,25 @@ __global__ void __launch_bounds__(192, 2)
   } else {
     // ------------------------------------------------------------ softmax warps 0-3
     const int row = threadIdx.x;  // TMEM lane == query row within the tile
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t tSrow = tS + ((uint32_t)(warp * 32) << 16);  // this warp's lane quarter
+    const uint32_t tOrow = tO + ((uint32_t)(warp * 32) << 16);
     const float sl2 = args.scale_log2;
     float m_used = -INFINITY;  // maximum the stored P and O are relative to (log2 domain)
     float l = 0.f;
-    bool whole = true;  // this CTA holds the item from its first key tile
-    uint8_t* prow0 = sP + row * 128;
-    int X = (int)(w0 / nt), j = (int)(w0 % nt);
-    for (int t = 0; t < T; ++t, j = (j + 1 == nt) ? 0 : j + 1, X += (j == 0)) {
+    const uint32_t prow0 = smem_u32(sP) + row * 128;  // this row of P, 32-bit shared address
+    int j = (int)(w0 % nt);  // key tile of step t within its item
+    for (int t = 0; t < T; ++t, j = (j + 1 == nt) ? 0 : j + 1) {
       const bool first = t == 0 || j == 0;
       const bool last = t == T - 1 || j == nt - 1;
-      if (first) whole = j == 0;
       if (!mbar_wait(s_full, t & 1, abort_flag, args.err)) break;
       tc_fence_after();
       const int kvalid = args.Nk - j * kAK;  // keys of this tile that exist
       // the whole S row into registers, then hand the TMEM columns back for S_{t+1}
       uint32_t sv[128];
-      tmem_ld_32x32b_x32(tS + lane_off + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld_32x32b_x32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_ld_32x32b_x32(tS + lane_off + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-      tmem_ld_32x32b_x32(tS + lane_off + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+      tmem_ld_32x32b_x32(tSrow + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld_32x32b_x32(tSrow + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld_32x32b_x32(tSrow + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+      tmem_ld_32x32b_x32(tSrow + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(s_free);
@@ -306,11 +351,11 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll 1
           for (int c = 0; c < 2; ++c) {
             uint32_t r[32];
-            tmem_ld_32x32b_x32(tO + lane_off + c * 32, r);
+            tmem_ld_32x32b_x32(tOrow + c * 32, r);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st_32x32b_x32(tO + lane_off + c * 32, r);
+            tmem_st_32x32b_x32(tOrow + c * 32, r);
           }
           tmem_st_wait();
           m_used = m_new;
@@ -328,11 +373,13 @@ __global__ void __launch_bounds__(192, 2)
           pk[i] = pack_bf16x2_alu(p0, p1);
         }
         // keys c*32 .. c*32+31 = half c/2, 16-byte chunks 4*(c&1) .. +3, swizzled by row
-        uint8_t* hrow = prow0 + (c >> 1) * kTileBytes;
+        const uint32_t hrow = prow0 + (c >> 1) * kTileBytes;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int chunk = ((c & 1) * 4 + q) ^ (row & 7);
-          *reinterpret_cast<uint4*>(hrow + chunk * 16) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(hrow + chunk * 16), "r"(pk[4 * q]),
+                       "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+                       : "memory");
         }
       }
       fence_proxy_async_smem();
@@ -343,47 +390,12 @@ __global__ void __launch_bounds__(192, 2)
       // ---------------------------------------------------------- end of this CTA's part of item X
       if (!mbar_wait(pv_done, t & 1, abort_flag, args.err)) break;
       tc_fence_after();
-      const int h = X / args.qtiles;
-      const int qrow = (X % args.qtiles) * kAQ + row;
-      __nv_bfloat16* dst = args.O + (size_t)qrow * args.ldo + h * 64;
-      if (whole && j == nt - 1) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tO + lane_off + c * 32, r);
-          tmem_ld_wait();
-          if (qrow < args.Nq) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              d4[u] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * u]) * inv, __uint_as_float(r[8 * u + 1]) * inv),
-                                 pack_bf16x2(__uint_as_float(r[8 * u + 2]) * inv, __uint_as_float(r[8 * u + 3]) * inv),
-                                 pack_bf16x2(__uint_as_float(r[8 * u + 4]) * inv, __uint_as_float(r[8 * u + 5]) * inv),
-                                 pack_bf16x2(__uint_as_float(r[8 * u + 6]) * inv, __uint_as_float(r[8 * u + 7]) * inv));
-            }
-          }
-        }
-        tc_fence_before();
-        continue;
-      }
-      // a piece of a split item: leave it in this CTA's slot (0 for its first item, 1 otherwise)
-      // for the merge kernel that runs after this one
-      float* slot = args.partial + ((size_t)blockIdx.x * 2 + (X == (int)(w0 / nt) ? 0 : 1)) * kSlotFloats;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tO + lane_off + c * 32, r);
-        tmem_ld_wait();
-        float4* o4 = reinterpret_cast<float4*>(slot + row * 64 + c * 32);
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          __stcg(o4 + u, make_float4(__uint_as_float(r[4 * u]), __uint_as_float(r[4 * u + 1]),
-                                     __uint_as_float(r[4 * u + 2]), __uint_as_float(r[4 * u + 3])));
+      {
+        const int w_first = (int)cta_first_step(blockIdx.x, args.steps, args.ctas);  // recomputed: rarely needed
+        attn_item_end(args, tOrow, row, (w_first + t) / nt, t >= j && j == nt - 1, (w_first + t) / nt == w_first / nt,
+                      m_used, l);
       }
       tc_fence_before();
-      __stcg(slot + 8192 + row, m_used);
-      __stcg(slot + 8320 + row, l);
     }
   }
 
@@ -396,55 +408,77 @@ __global__ void __launch_bounds__(192, 2)
 // Merge of split items: block b looks at the boundary between CTAs b and b+1;
 // if it falls inside an item and is that item's first boundary, the block
 // merges the item's pieces in CTA order: M = max m_p, O = sum 2^(m_p - M) O_p /
-// sum 2^(m_p - M) l_p. Two threads per query row, 32 output columns each.
-__global__ void __launch_bounds__(256) attention_merge_kernel(const __grid_constant__ AttnArgs args) {
+// sum 2^(m_p - M) l_p. Four threads per query row, 16 output columns each; up to
+// kMergeBatch pieces are loaded before any is used.
+constexpr int kMergeBatch = 4;
+
+__global__ void __launch_bounds__(512) attention_merge_kernel(const __grid_constant__ AttnArgs args) {
   pdl_wait();
   pdl_trigger();
   const int nt = args.ktiles;
   const int64_t b = blockIdx.x + 1;
   const int64_t s0 = cta_first_step(b, args.steps, args.ctas);
-  if (s0 % nt == 0) return;                                            // boundary between items
-  if (cta_first_step(b - 1, args.steps, args.ctas) / nt == s0 / nt &&
-      cta_first_step(b - 1, args.steps, args.ctas) % nt != 0)
-    return;                                                            // an earlier boundary merges it
+  if (s0 % nt == 0) return;  // boundary between items
+  const int64_t sprev = cta_first_step(b - 1, args.steps, args.ctas);
+  if (sprev / nt == s0 / nt && sprev % nt != 0) return;  // an earlier boundary merges this item
   const int X = (int)(s0 / nt);
-  const int64_t s_lo = (int64_t)X * nt, s_hi = s_lo + nt - 1;
-  int64_t c_lo = b - 1, c_hi = b;
+  const int64_t s_hi = (int64_t)X * nt + nt - 1;
+  const int64_t c_lo = b - 1;
+  int64_t c_hi = b;
   while (c_hi + 1 < args.ctas && cta_first_step(c_hi + 1, args.steps, args.ctas) <= s_hi) ++c_hi;
-  (void)s_lo;
-  const int row = threadIdx.x >> 1, half = threadIdx.x & 1;
-  float mmax = -INFINITY;
-  for (int64_t c = c_lo; c <= c_hi; ++c) {
-    const int fi = (int)(cta_first_step(c, args.steps, args.ctas) / nt);
-    const float* sl = args.partial + ((size_t)c * 2 + (X == fi ? 0 : 1)) * kSlotFloats;
-    mmax = fmaxf(mmax, __ldcg(sl + 8192 + row));
-  }
-  float acc[32];
+  const int row = threadIdx.x >> 2, quarter = threadIdx.x & 3;
+  float mmax = -INFINITY, lsum = 0.f;
+  float acc[16];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-  float lsum = 0.f;
-  for (int64_t c = c_lo; c <= c_hi; ++c) {
-    const int fi = (int)(cta_first_step(c, args.steps, args.ctas) / nt);
-    const float* sl = args.partial + ((size_t)c * 2 + (X == fi ? 0 : 1)) * kSlotFloats;
-    const float e = ex2(__ldcg(sl + 8192 + row) - mmax);
-    lsum += e * __ldcg(sl + 8320 + row);
-    const float4* o4 = reinterpret_cast<const float4*>(sl + row * 64 + half * 32);
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  for (int64_t c0 = c_lo; c0 <= c_hi; c0 += kMergeBatch) {
+    float m[kMergeBatch], l[kMergeBatch];
+    float4 o[kMergeBatch][4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float4 v = __ldcg(o4 + u);
-      acc[4 * u] += e * v.x;
-      acc[4 * u + 1] += e * v.y;
-      acc[4 * u + 2] += e * v.z;
-      acc[4 * u + 3] += e * v.w;
+    for (int p = 0; p < kMergeBatch; ++p) {
+      const int64_t c = c0 + p;
+      m[p] = -INFINITY;
+      l[p] = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) o[p][u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c <= c_hi) {
+        const int fi = (int)(cta_first_step(c, args.steps, args.ctas) / nt);
+        const float* sl = args.partial + ((size_t)c * 2 + (X == fi ? 0 : 1)) * kSlotFloats;
+        m[p] = __ldcg(sl + 8192 + row);
+        l[p] = __ldcg(sl + 8320 + row);
+        const float4* o4 = reinterpret_cast<const float4*>(sl + row * 64 + quarter * 16);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) o[p][u] = __ldcg(o4 + u);
+      }
     }
+    float mb = mmax;
+#pragma unroll
+    for (int p = 0; p < kMergeBatch; ++p) mb = fmaxf(mb, m[p]);
+    const float rescale = mmax == -INFINITY ? 0.f : ex2(mmax - mb);  // earlier batches to the new maximum
+    lsum *= rescale;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] *= rescale;
+#pragma unroll
+    for (int p = 0; p < kMergeBatch; ++p) {
+      const float e = m[p] == -INFINITY ? 0.f : ex2(m[p] - mb);
+      lsum += e * l[p];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[4 * u] += e * o[p][u].x;
+        acc[4 * u + 1] += e * o[p][u].y;
+        acc[4 * u + 2] += e * o[p][u].z;
+        acc[4 * u + 3] += e * o[p][u].w;
+      }
+    }
+    mmax = mb;
   }
   const int h = X / args.qtiles;
   const int qrow = (X % args.qtiles) * kAQ + row;
   if (qrow >= args.Nq) return;
   const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-  uint4* d4 = reinterpret_cast<uint4*>(args.O + (size_t)qrow * args.ldo + h * 64 + half * 32);
+  uint4* d4 = reinterpret_cast<uint4*>(args.O + (size_t)qrow * args.ldo + h * 64 + quarter * 16);
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
+  for (int u = 0; u < 2; ++u)
     d4[u] = make_uint4(pack_bf16x2(acc[8 * u] * inv, acc[8 * u + 1] * inv),
                        pack_bf16x2(acc[8 * u + 2] * inv, acc[8 * u + 3] * inv),
                        pack_bf16x2(acc[8 * u + 4] * inv, acc[8 * u + 5] * inv),
@@ -455,13 +489,13 @@ size_t attention_partial_bytes(int num_sms) { return (size_t)2 * num_sms * 2 * k
 
 // Split the key tiles of items between CTAs only when that shortens the
 // longest CTA: with whole items a CTA alone on its SM runs a step in about 0.6
-// of the time two co-resident CTAs take; a split adds about two steps of
-// overhead (the pieces and their merge).
+// of the time two co-resident CTAs take; a split costs about ten steps (the
+// extra Q loads and pipeline fills of the pieces and the merge kernel).
 static bool attention_split_pays(int items, int ktiles, int num_sms) {
   if (ktiles < 2) return false;
   const int resident = 2 * num_sms;
   const double whole = items <= num_sms ? 0.6 * ktiles : (double)((items + resident - 1) / resident) * ktiles;
-  const double split = (double)items * ktiles / resident + 2.0;
+  const double split = (double)items * ktiles / resident + 10.0;
   return split < whole;
 }
 
@@ -507,7 +541,7 @@ int launch_attention_tc(const __nv_bfloat16* qbase, int q_ld, int q_rows, int q_
   }
   int e = (int)launch_pdl(attention_tc_kernel, dim3(a.ctas), dim3(192), smem, st, maps, a);
   if (e != 0 || !split || a.ctas < 2) return e;
-  return (int)launch_pdl(attention_merge_kernel, dim3(a.ctas - 1), dim3(256), 0, st, a);
+  return (int)launch_pdl(attention_merge_kernel, dim3(a.ctas - 1), dim3(512), 0, st, a);
 }
 
 }  // namespace sdk

@@ -135,9 +135,9 @@ TX_CASES = [
     (8, 8, 640, 2, 2048, 77, True),
     (16, 16, 256, 1, 256, 5, False),
     (4, 6, 1280, 1, 2048, 77, False),
-    # 180 (head, query tile) items of 18 key tiles: the self-attention key tiles are
-    # spread over all CTAs and split items are merged by the second kernel
-    (48, 48, 640, 1, 1024, 77, False),
+    # 320 (head, query tile) items of 32 key tiles: the self-attention key tiles are
+    # spread evenly over all CTAs and split items are merged by the second kernel
+    (64, 64, 640, 1, 1024, 77, False),
 ]
 
 
