@@ -125,6 +125,28 @@ class ClockSampler:
 MID_PREFIXES = ("mid.", "time.")
 
 
+def measured_traffic(kernel):
+    """DRAM bytes per launch of ``kernel`` from the committed ncu summary, or None
+    when there is none or the kernel's source changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel}_dram_traffic_unet_step_sd21_96.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.split(":", 1)[0] in ("traffic_bytes_per_launch", "source", "source_sha256"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    try:
+        src = os.path.join(ROOT, fields["source"])
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if digest != fields["source_sha256"]:
+            return None
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, OSError, ValueError):
+        return None
+
+
 def mid_params(seed=4, canonical_unet=None):
     """Oracle parameters of the time MLP and the mid block of the SD2.1-base
     U-Net: sliced from the canonical buffer when given, else drawn from the
@@ -213,6 +235,24 @@ def cpu_cores():
 
 
 # ----------------------------------------------------------------------------- reference arm
+
+def slowest_rank_ms(ms, world, device=None):
+    """Per-step time of the slowest rank (max over ranks); the local value for one rank.
+    Every rank must call it at the same point (it is a collective for world > 1)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_steps_per_s(ms_step, world):
+    """Whole-job throughput of `world` independent replicas, each timed by the slowest rank."""
+    return world * 1e3 / ms_step
+
 
 def run_reference(args, rank, world):
     """The oracle as the reference arm: every step is the bounded mid-block
@@ -337,11 +377,8 @@ def main():
     ms_step = ms_total / args.steps
     # graph replays do not pass through the host library: every replay launches the captured kernels
     gpu_launches = n_graph * args.steps + (B.sd_launch_count() - launches_before)
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = world * 1e3 / ms_step
+    ms_step = slowest_rank_ms(ms_step, world, dev)
+    value = aggregate_steps_per_s(ms_step, world)
     tflops = step_flops / (ms_step * 1e-3) / 1e12
 
     # second timed region: the same step with an event pair around every launch
@@ -378,7 +415,9 @@ def main():
         achieved = dom["flops"] / dom["launches"] / (avg_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roof = {"kernel": dom_name, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": measured_traffic(dom_name),
+                "traffic_unit": "bytes per launch (ncu dram read + write, committed summary)",
+                "algorithmic_bytes_per_launch": dom["bytes"] / dom["launches"],
                 "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
                 "launches_per_step": dom["launches"], "avg_launch_us": avg_ms * 1e3,
                 "algorithmic_flops_per_launch": dom["flops"] / dom["launches"],
@@ -419,11 +458,8 @@ def main():
     torch.cuda.synchronize(dev)
     wall = time.perf_counter() - t_wall
     e2e_ms = max(e0.elapsed_time(e1), wall * 1e3) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * 1e3 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": lat_h.numel() * 2 + ctx_h.numel() * 2,
+    e2e_ms = slowest_rank_ms(e2e_ms, world, dev)
+    e2e = {"value": aggregate_steps_per_s(e2e_ms, world), "unit": UNIT, "h2d_bytes_per_step": lat_h.numel() * 2 + ctx_h.numel() * 2,
            "d2h_bytes_per_step": eps_h.numel() * 2, "ms_per_step": e2e_ms,
            "path": "pinned host latent+context -> device, sd_unet_step (eager ABI call), eps -> pinned host, "
                    "stream synchronised every step"}

@@ -61,8 +61,4 @@ int launch_attention_tc(const __nv_bfloat16* qbase, int q_ld, int q_rows, int q_
                         int kv_ld, int kv_rows, int k_col, int v_col, __nv_bfloat16* O, int ldo, int Nq, int Nk,
                         int heads, float* partial, size_t partial_bytes, int num_sms, int* err, cudaStream_t st);
 
-// Flash attention (head_dim 64) on mma.sync: O[i, h*64 + d] = softmax_j(Q_i.K_j / 8) V_j per head.
-int launch_attention(const __nv_bfloat16* Q, int ldq, const __nv_bfloat16* K, int ldk, const __nv_bfloat16* V,
-                     int ldv, __nv_bfloat16* O, int ldo, int Nq, int Nk, int heads, cudaStream_t st);
-
 }  // namespace sdk

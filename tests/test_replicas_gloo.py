@@ -1,0 +1,62 @@
+"""The multi-GPU path of bench.py is N independent replicas: the only
+cross-rank steps are the barrier and the max-reduction of the per-step time.
+Those run here as two gloo ranks on CPU (no GPU), and the reference arm's
+non-zero ranks must return without work."""
+import os
+import socket
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist  # noqa: E402
+import torch.multiprocessing as mp  # noqa: E402
+
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    from datetime import timedelta
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        local = 5.0 + 1.25 * rank  # rank 1 is the slower replica
+        ms = bench.slowest_rank_ms(local, world)
+        e2e = bench.slowest_rank_ms(10.0 - rank, world)  # here rank 0 is the slower one
+        dist.barrier()
+        out[rank] = (ms, e2e, bench.aggregate_steps_per_s(ms, world))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_time():
+    world = 2
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    assert set(res) == {0, 1}
+    for rank in (0, 1):
+        ms, e2e, value = res[rank]
+        assert ms == 6.25 and e2e == 10.0
+        assert value == pytest.approx(2 * 1e3 / 6.25)
+
+
+def test_single_rank_needs_no_process_group():
+    assert not dist.is_initialized()
+    assert bench.slowest_rank_ms(4.0, 1) == 4.0
+    assert bench.aggregate_steps_per_s(4.0, 1) == 250.0
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    class Args:
+        steps, warmup = 1, 0
+
+    assert bench.run_reference(Args, rank=1, world=2) == 0
