@@ -10,6 +10,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "gemm_tc.cuh"
@@ -80,17 +81,29 @@ struct Ctx {
   size_t skws_bytes;
   float* attn_part;   // pieces of split attention items
   size_t attn_part_bytes;
+  // two row-statistics buffers of [rs_rows][2] for the folded LayerNorms (zeroed every call);
+  // *rs_clean is the host's record of the one that is zero now
+  unsigned long long* rs[2];
+  int64_t rs_rows;
+  int* rs_clean;
+  size_t clear_bytes;  // header, GroupNorm accumulators and row statistics: one memset per call
   int sms;
 };
 
 constexpr size_t kSplitKBytes = size_t(16) << 20;
 
-// Header + GroupNorm scratch at the start of every workspace.
-Ctx make_ctx(Arena& ar, cudaStream_t st, int sms) {
+// Header + GroupNorm scratch (+ row statistics for `rs_rows` tokens) at the start of every workspace.
+Ctx make_ctx(Arena& ar, cudaStream_t st, int sms, int64_t rs_rows = 0) {
   Ctx c;
-  uint8_t* h = static_cast<uint8_t*>(ar.take(kHeaderBytes + kGnAccBytes));
+  const size_t rs_bytes = (size_t)rs_rows * 2 * sizeof(unsigned long long);
+  c.clear_bytes = kHeaderBytes + kGnAccBytes + 2 * rs_bytes;
+  uint8_t* h = static_cast<uint8_t*>(ar.take(c.clear_bytes));
   c.err = reinterpret_cast<int*>(h);
   c.gn_acc = h ? reinterpret_cast<unsigned long long*>(h + kHeaderBytes) : nullptr;
+  c.rs_rows = rs_rows;
+  c.rs[0] = h && rs_rows ? reinterpret_cast<unsigned long long*>(h + kHeaderBytes + kGnAccBytes) : nullptr;
+  c.rs[1] = c.rs[0] ? c.rs[0] + rs_rows * 2 : nullptr;
+  c.rs_clean = nullptr;
   c.gn_seq = nullptr;
   c.skws = static_cast<float*>(ar.take(kSplitKBytes));
   c.skws_bytes = kSplitKBytes;
@@ -180,9 +193,24 @@ void add_conv3x3_segs(GemmProblem& p, int amap, int bmap, int C) {
 }
 
 // y[M, N] = A[M, K] B[N, K]^T (+ epilogue), A a token matrix.
+// LayerNorm folded into a linear layer. A producer GEMM adds its output rows'
+// sums into `out` and zeroes `clear`; a consumer GEMM reads the raw LayerNorm
+// input as A, its row sums from `in`, and the column terms c1 / c2 of B packed
+// as W * gamma.
+struct LnFold {
+  unsigned long long* out = nullptr;
+  unsigned long long* clear = nullptr;
+  int64_t clear_elems = 0;
+  const unsigned long long* in = nullptr;
+  const float* c1 = nullptr;
+  const float* c2 = nullptr;
+  int cols = 0;
+  float eps = 0.f;
+};
+
 sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, int N, const bf16* bias,
                      const bf16* residual, int ld_res, bf16* out, int ld_out, int mode = sdk::GEMM_PLAIN,
-                     double alg_k = 0, int f16_begin = 0) {
+                     double alg_k = 0, int f16_begin = 0, const LnFold* ln = nullptr) {
   GemmProblem p = base_problem(c);
   p.Ho = 1;
   p.Wo = M;
@@ -200,6 +228,16 @@ sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, i
   p.epi.ld_out = ld_out;
   p.epi.mode = mode;
   p.epi.f16_begin = f16_begin;
+  if (ln) {
+    p.epi.rowstat_out = ln->out;
+    p.epi.rowstat_clear = ln->clear;
+    p.epi.rowstat_clear_elems = ln->clear_elems;
+    p.epi.rowstat_in = ln->in;
+    p.epi.colscale = ln->c1;
+    if (ln->in) p.epi.colvec = ln->c2;
+    p.epi.ln_cols = ln->cols;
+    p.epi.ln_eps = ln->eps;
+  }
   CK(launch_gemm(c, p, alg_k));
   return SD_OK;
 }
@@ -310,11 +348,6 @@ TxScratch plan_tx_scratch(Arena& ar, int HW, int C, int ctx_len) {
   return s;
 }
 
-int run_ln(const Ctx& c, const bf16* x, int N, int C, const bf16* g, const bf16* b, float eps, bf16* y) {
-  sdp::Scope sc("layernorm", sdp::F_LN, 0, 4.0 * N * C, c.st);
-  return sdk::launch_layernorm(x, N, C, g, b, eps, y, c.st);
-}
-
 // Attention of Q (rows of qbase, columns q_col + 64h) against K/V (rows of
 // kvbase, columns k_col + 64h and v_col + 64h), head_dim 64, into O [Nq, ldo].
 int run_attn(const Ctx& c, const bf16* qbase, int q_ld, int q_col, const bf16* kvbase, int kv_ld, int k_col,
@@ -332,29 +365,91 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
   const int HW = H * Wd;
   const int C = w.C;
   const int heads = C / 64;
+  if (!c.rs[0] || !c.rs_clean || c.rs_rows < HW) return SD_ERR_UNSUPPORTED;
+  // The three LayerNorms of each block are folded into the GEMMs they feed
+  // (Q/K/V, the cross-attention query, FF1): every GEMM that writes the
+  // residual stream t also leaves t's row sums in one of two buffers, and
+  // zeroes the other one, whose last reader ran before it.
+  int cur = -1;              // buffer holding the row sums of t
+  int clean = *c.rs_clean;  // buffer that is zero
+  auto producer = [&]() {
+    LnFold f;
+    f.out = c.rs[clean];
+    f.clear = cur >= 0 ? c.rs[cur] : nullptr;
+    f.clear_elems = c.rs_rows * 2;
+    if (cur >= 0) {
+      std::swap(cur, clean);
+    } else {
+      cur = clean;
+      clean = 1 - clean;
+    }
+    return f;
+  };
+  auto consumer = [&](int64_t c1, int64_t c2) {
+    LnFold f;
+    f.in = c.rs[cur];
+    f.c1 = reinterpret_cast<const float*>(static_cast<const uint8_t*>(pw) + c1);
+    f.c2 = reinterpret_cast<const float*>(static_cast<const uint8_t*>(pw) + c2);
+    f.cols = C;
+    f.eps = ln_eps;
+    return f;
+  };
   sd_status r;
   if ((r = run_gn(c, x, C, nullptr, 0, HW, G, gn_eps, W(pw, w.ng), W(pw, w.nb), 0, s.nrm)) != SD_OK) return r;
-  if ((r = run_linear(c, s.nrm, HW, C, W(pw, w.piw), C, W(pw, w.pib), nullptr, 0, s.t, C)) != SD_OK) return r;
+  {
+    // the other buffer is not known to be zero yet: clear it too
+    LnFold f = producer();
+    f.clear = c.rs[clean];
+    if ((r = run_linear(c, s.nrm, HW, C, W(pw, w.piw), C, W(pw, w.pib), nullptr, 0, s.t, C, sdk::GEMM_PLAIN, 0, 0,
+                        &f)) != SD_OK)
+      return r;
+  }
   for (const TxBlockW& b : w.blocks) {
-    // self-attention: t += Wo Attn(LN1(t))
-    CK(run_ln(c, s.t, HW, C, W(pw, b.ln1g), W(pw, b.ln1b), ln_eps, s.nrm));
-    if ((r = run_linear(c, s.nrm, HW, C, W(pw, b.qkv), 3 * C, nullptr, nullptr, 0, s.big, 3 * C)) != SD_OK) return r;
+    // self-attention: t += Wo Attn(LN1(t)), LN1 folded into the Q/K/V GEMM
+    {
+      const LnFold f = consumer(b.qkv_c1, b.qkv_c2);
+      if ((r = run_linear(c, s.t, HW, C, W(pw, b.qkv), 3 * C, nullptr, nullptr, 0, s.big, 3 * C, sdk::GEMM_PLAIN, 0,
+                          0, &f)) != SD_OK)
+        return r;
+    }
     CK(run_attn(c, s.big, 3 * C, 0, s.big, 3 * C, C, 2 * C, s.ao, C, HW, HW, heads));
-    if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o1w), C, W(pw, b.o1b), s.t, C, s.t, C)) != SD_OK) return r;
+    {
+      const LnFold f = producer();
+      if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o1w), C, W(pw, b.o1b), s.t, C, s.t, C, sdk::GEMM_PLAIN, 0, 0,
+                          &f)) != SD_OK)
+        return r;
+    }
     // cross-attention: t += Wo' Attn(LN2(t), ctx)
-    CK(run_ln(c, s.t, HW, C, W(pw, b.ln2g), W(pw, b.ln2b), ln_eps, s.nrm));
-    if ((r = run_linear(c, s.nrm, HW, C, W(pw, b.q2), C, nullptr, nullptr, 0, s.big, C)) != SD_OK) return r;
+    {
+      const LnFold f = consumer(b.q2_c1, b.q2_c2);
+      if ((r = run_linear(c, s.t, HW, C, W(pw, b.q2), C, nullptr, nullptr, 0, s.big, C, sdk::GEMM_PLAIN, 0, 0, &f)) !=
+          SD_OK)
+        return r;
+    }
     if ((r = run_linear(c, ctx, ctx_len, w.ctx_dim, W(pw, b.kv2), 2 * C, nullptr, nullptr, 0, s.kv, 2 * C)) != SD_OK)
       return r;
     CK(run_attn(c, s.big, C, 0, s.kv, 2 * C, 0, C, s.ao, C, HW, ctx_len, heads));
-    if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o2w), C, W(pw, b.o2b), s.t, C, s.t, C)) != SD_OK) return r;
-    // GEGLU feed-forward: t += W2 (a * GELU(g)) + b2
-    CK(run_ln(c, s.t, HW, C, W(pw, b.ln3g), W(pw, b.ln3b), ln_eps, s.nrm));
-    if ((r = run_linear(c, s.nrm, HW, C, W(pw, b.f1w), 8 * C, W(pw, b.f1b), nullptr, 0, s.big, 4 * C,
-                        sdk::GEMM_GEGLU)) != SD_OK)
-      return r;
-    if ((r = run_linear(c, s.big, HW, 4 * C, W(pw, b.f2w), C, W(pw, b.f2b), s.t, C, s.t, C)) != SD_OK) return r;
+    {
+      const LnFold f = producer();
+      if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o2w), C, W(pw, b.o2b), s.t, C, s.t, C, sdk::GEMM_PLAIN, 0, 0,
+                          &f)) != SD_OK)
+        return r;
+    }
+    // GEGLU feed-forward: t += W2 (a * GELU(g)) + b2, LN3 folded into FF1 (its bias is in c2)
+    {
+      const LnFold f = consumer(b.f1_c1, b.f1_c2);
+      if ((r = run_linear(c, s.t, HW, C, W(pw, b.f1w), 8 * C, nullptr, nullptr, 0, s.big, 4 * C, sdk::GEMM_GEGLU, 0,
+                          0, &f)) != SD_OK)
+        return r;
+    }
+    {
+      const LnFold f = producer();
+      if ((r = run_linear(c, s.big, HW, 4 * C, W(pw, b.f2w), C, W(pw, b.f2b), s.t, C, s.t, C, sdk::GEMM_PLAIN, 0, 0,
+                          &f)) != SD_OK)
+        return r;
+    }
   }
+  *c.rs_clean = clean;
   // y = x + proj_out(t)
   return run_linear(c, s.t, HW, C, W(pw, w.pow_), C, W(pw, w.pob), x, C, y, C);
 }
@@ -533,7 +628,7 @@ struct TxPlan {
   TxScratch s;
 };
 size_t plan_tx(Arena& ar, const sd_transformer_cfg* cfg, cudaStream_t st, int sms, TxPlan* p) {
-  p->c = make_ctx(ar, st, sms);
+  p->c = make_ctx(ar, st, sms, (int64_t)cfg->height * cfg->width);
   p->s = plan_tx_scratch(ar, cfg->height * cfg->width, cfg->channels, cfg->ctx_len);
   return ar.off;
 }
@@ -581,7 +676,7 @@ struct UNetPlan {
 size_t plan_unet(Arena& ar, const sd_unet_cfg* cfg, cudaStream_t st, int sms, UNetPlan* p) {
   const int L = cfg->n_levels;
   const int* ch = cfg->block_channels;
-  p->c = make_ctx(ar, st, sms);
+  p->c = make_ctx(ar, st, sms, (int64_t)cfg->height * cfg->width);  // the largest level
   p->phi = ar.f32(cfg->time_proj_dim);
   p->hid = ar.f32(cfg->temb_dim);
   p->temb = ar.f32(cfg->temb_dim);
@@ -685,7 +780,7 @@ sd_status check_ws(size_t need, const void* ws, size_t ws_bytes) {
 
 // Zero the device error word and this call's GroupNorm accumulators.
 sd_status clear_header(const Ctx& c) {
-  if (cudaMemsetAsync(c.err, 0, kHeaderBytes + kGnAccBytes, c.st) != cudaSuccess) return SD_ERR_LAUNCH;
+  if (cudaMemsetAsync(c.err, 0, c.clear_bytes, c.st) != cudaSuccess) return SD_ERR_LAUNCH;
   return SD_OK;
 }
 
@@ -873,6 +968,8 @@ sd_status sd_time_embed(const sd_time_cfg* cfg, const void* pw, float timestep, 
   if ((s = clear_header(p.c)) != SD_OK) return s;
   int gn_seq = 0;
   p.c.gn_seq = &gn_seq;
+  int rs_clean = 0;  // both row-statistics buffers are zeroed with the header
+  p.c.rs_clean = &rs_clean;
   Table tab;
   TimeW w = add_time(tab, "time", cfg->proj_dim, cfg->temb_dim);
   return run_time(p.c, w, pw, cfg->proj_dim, cfg->temb_dim, timestep, p.phi, p.hid, temb);
@@ -896,6 +993,8 @@ sd_status sd_conv_fwd(const sd_conv_cfg* cfg, int32_t kind, const void* pw, cons
   if ((s = clear_header(p.c)) != SD_OK) return s;
   int gn_seq = 0;
   p.c.gn_seq = &gn_seq;
+  int rs_clean = 0;  // both row-statistics buffers are zeroed with the header
+  p.c.rs_clean = &rs_clean;
   Table tab;
   const int H = cfg->height, Wd = cfg->width;
   const bf16* X0 = static_cast<const bf16*>(x0);
@@ -940,6 +1039,8 @@ sd_status sd_resblock_fwd(const sd_resblock_cfg* cfg, const void* pw, const void
   if ((s = clear_header(p.c)) != SD_OK) return s;
   int gn_seq = 0;
   p.c.gn_seq = &gn_seq;
+  int rs_clean = 0;  // both row-statistics buffers are zeroed with the header
+  p.c.rs_clean = &rs_clean;
   Table tab;
   ResW w = add_resblock(tab, "res", cfg->c_x + cfg->c_skip, cfg->c_out, cfg->temb_dim);
   sdk::GemvBatch b;
@@ -970,6 +1071,8 @@ sd_status sd_transformer_fwd(const sd_transformer_cfg* cfg, const void* pw, cons
   if ((s = clear_header(p.c)) != SD_OK) return s;
   int gn_seq = 0;
   p.c.gn_seq = &gn_seq;
+  int rs_clean = 0;  // both row-statistics buffers are zeroed with the header
+  p.c.rs_clean = &rs_clean;
   Table tab;
   TxW w = add_transformer(tab, "attn", cfg->channels, cfg->depth, cfg->ctx_dim);
   return run_transformer(p.c, w, pw, cfg->height, cfg->width, static_cast<const bf16*>(x),
@@ -993,6 +1096,8 @@ sd_status sd_unet_step(const sd_unet_cfg* cfg, const void* pw, const void* laten
   if ((s = clear_header(c)) != SD_OK) return s;
   int gn_seq = 0;
   p.c.gn_seq = &gn_seq;
+  int rs_clean = 0;  // both row-statistics buffers are zeroed with the header
+  p.c.rs_clean = &rs_clean;
   Table tab;
   UNetW u = add_unet(tab, *cfg);
   const int L = cfg->n_levels;

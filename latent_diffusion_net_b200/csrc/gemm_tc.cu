@@ -24,7 +24,7 @@ constexpr int kGemmThreads = 64 + kEpiThreads;
 
 constexpr int kMaxStages = 12;
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA on sm_100
-constexpr int kSmemFixed = 1024 + 256 + 2048;  // alignment slack, barriers, per-column terms
+constexpr int kSmemFixed = 1024 + 256 + 4096;  // alignment slack, barriers, per-column terms (2 x [2][256])
 
 struct __align__(64) GemmMaps {
   CUtensorMap a[kGemmMaxA];   // BH x BW pixel boxes
@@ -153,7 +153,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_empty = acc_full + 2;       // [2], used in the even CTA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* epi_col = reinterpret_cast<float*>(smem + STAGES * stage_bytes + 256);  // [2][256]
+  float* epi_col = reinterpret_cast<float*>(smem + STAGES * stage_bytes + 256);  // [2][256] added terms
+  float* epi_scl = epi_col + 512;                                                // [2][256] LayerNorm colscale
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -181,6 +182,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // everything above touched only shared memory and TMEM: wait for the previous kernel here
   pdl_wait();
   pdl_trigger();
+  if (args.epi.rowstat_clear) {
+    // every kernel before this one has finished: the buffer's last reader among them
+    const int64_t n2 = args.epi.rowstat_clear_elems / 2;
+    ulonglong2* z = reinterpret_cast<ulonglong2*>(args.epi.rowstat_clear);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += (int64_t)gridDim.x * blockDim.x)
+      z[i] = make_ulonglong2(0ull, 0ull);
+  }
 
   if (warp == 0) {
     if (lane == 0) {
@@ -313,6 +321,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const bool geglu = args.epi.mode == GEMM_GEGLU;
     __nv_bfloat16* const out = args.epi.out;
     const bool has_cols = partial == nullptr && (bias || bias2 || colvec);
+    unsigned long long* const rowstat_out = args.epi.rowstat_out;
+    const unsigned long long* const rowstat_in = partial ? nullptr : args.epi.rowstat_in;
+    const float* const colscale = args.epi.colscale;
+    const double ln_inv = args.epi.ln_cols > 0 ? 1.0 / args.epi.ln_cols : 0.0;
+    const float ln_eps = args.epi.ln_eps;
 
     const int et = threadIdx.x - 64;  // 0..255
     const int half = (warp - 2) >> 2;  // which alternate 32-column chunks this warp handles
@@ -330,6 +343,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int n0 = nt * BN;
       const int b = it & 1;
       float* const ecol = epi_col + b * 256;
+      float* const escl = epi_scl + b * 256;
+      if (rowstat_in) {
+        for (int c = et; c < BN; c += kEpiThreads) {
+          const int n = n0 + c;
+          escl[c] = n < N ? colscale[n] : 0.f;
+        }
+        if (!has_cols) asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
+      }
       if (has_cols) {
         // per-column terms of this unit (biases + FP32 column vector), computed
         // while the main loop runs; buffer b was last read two units ago
@@ -345,12 +366,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
       }
-      const bool have = mbar_wait(&acc_full[b], (it >> 1) & 1, abort_flag, args.err);
-      tc_fence_after();
       const int oy = (mt / tiles_x) * BH + row / BW;
       const int ox = (mt % tiles_x) * BW + row % BW;
-      const bool valid = have && mt < tiles_m && oy < Ho && ox < Wo;
+      const bool in_image = mt < tiles_m && oy < Ho && ox < Wo;
       const long grow = (long)oy * Wo + ox;
+      // LayerNorm of this row from its fixed-point sums (final before this kernel
+      // started), computed while the main loop runs: v = rstd*acc - rstd*mean*colscale + colvec
+      float ln_a = 1.f, ln_b = 0.f;
+      if (rowstat_in && in_image) {
+        const double s1 = (double)(long long)__ldcg(rowstat_in + 2 * grow) * (1.0 / kRowSumScale);
+        const double s2 = (double)(long long)__ldcg(rowstat_in + 2 * grow + 1) * (1.0 / kRowSqScale);
+        const double mean = s1 * ln_inv;
+        const double var = fmax(s2 * ln_inv - mean * mean, 0.0);
+        const float rstd = (float)(1.0 / sqrt(var + (double)ln_eps));
+        ln_a = rstd;
+        ln_b = (float)(-mean) * rstd;
+      }
+      const bool have = mbar_wait(&acc_full[b], (it >> 1) & 1, abort_flag, args.err);
+      tc_fence_after();
+      const bool valid = have && in_image;
+      float rs1 = 0.f, rs2 = 0.f;  // this thread's part of the row sums of the stored output
       const uint32_t tacc = tmem_base + (uint32_t)(b * 256) + lane_off;
       if (half >= kChunks) {
         // no chunk for this warp (BN = 32): still take part in the release
@@ -373,7 +408,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int nb = n0 + cc * 32;
         if (nb >= N) continue;
         float v[32];
-        if (has_cols) {
+        if (rowstat_in) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            v[j] = fmaf(ln_a, __uint_as_float(r[j]), fmaf(ln_b, escl[cc * 32 + j], has_cols ? ecol[cc * 32 + j] : 0.f));
+        } else if (has_cols) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + ecol[cc * 32 + j];
         } else {
@@ -456,11 +495,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             d4[w] = make_uint4(pack_bf16x2(v[8 * w + 0], v[8 * w + 1]), pack_bf16x2(v[8 * w + 2], v[8 * w + 3]),
                                pack_bf16x2(v[8 * w + 4], v[8 * w + 5]), pack_bf16x2(v[8 * w + 6], v[8 * w + 7]));
           }
+          if (rowstat_out) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float q = __bfloat162float(__float2bfloat16_rn(v[j]));
+              rs1 += q;
+              rs2 = fmaf(q, q, rs2);
+            }
+          }
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (nb + j < N) dst[j] = __float2bfloat16_rn(v[j]);
+          for (int j = 0; j < 32; ++j) {
+            if (nb + j < N) {
+              const __nv_bfloat16 q = __float2bfloat16_rn(v[j]);
+              dst[j] = q;
+              if (rowstat_out) {
+                rs1 += __bfloat162float(q);
+                rs2 = fmaf(__bfloat162float(q), __bfloat162float(q), rs2);
+              }
+            }
+          }
         }
+      }
+      if (rowstat_out && !partial && valid && half < kChunks) {
+        // integer adds: the sums do not depend on the order in which units arrive
+        atomicAdd(rowstat_out + 2 * grow, (unsigned long long)llrint((double)rs1 * kRowSumScale));
+        atomicAdd(rowstat_out + 2 * grow + 1, (unsigned long long)llrint((double)rs2 * kRowSqScale));
       }
     }
   }
@@ -472,51 +532,102 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_dealloc_2sm(tmem_base, kTmemCols);
 }
 
+// Split-K reduction of 8 columns (row, c .. c+7): sum over splits of the FP32
+// partials in split order (deterministic), then the epilogue. Returns, through
+// rs1 / rs2, the sums of the stored BF16 values (plain stores only).
+__device__ __forceinline__ void splitk_reduce_vec(const float* __restrict__ partial, int splits, int M, int N,
+                                                  const GemmEpi& epi, int row, int c, float& rs1, float& rs2) {
+  float v[8];
+  const float4* p0 = reinterpret_cast<const float4*>(partial + (size_t)row * N + c);
+  float4 a = p0[0], b = p0[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  for (int z = 1; z < splits; ++z) {
+    const float4* pz = reinterpret_cast<const float4*>(partial + ((size_t)z * M + row) * N + c);
+    a = pz[0];
+    b = pz[1];
+    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w; v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  }
+  if (epi.rowstat_in) {
+    // folded LayerNorm: rstd * acc - rstd * mean * colscale + colvec
+    const double s1 = (double)(long long)__ldcg(epi.rowstat_in + 2 * row) * (1.0 / kRowSumScale);
+    const double s2 = (double)(long long)__ldcg(epi.rowstat_in + 2 * row + 1) * (1.0 / kRowSqScale);
+    const double inv = 1.0 / epi.ln_cols;
+    const double mean = s1 * inv;
+    const double var = fmax(s2 * inv - mean * mean, 0.0);
+    const float rstd = (float)(1.0 / sqrt(var + (double)epi.ln_eps));
+    const float lb = (float)(-mean) * rstd;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = fmaf(rstd, v[j], lb * epi.colscale[c + j]);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float add = 0.f;
+    if (epi.bias) add += __bfloat162float(epi.bias[c + j]);
+    if (epi.bias2) add += __bfloat162float(epi.bias2[c + j]);
+    if (epi.colvec) add += epi.colvec[c + j];
+    v[j] += add;
+  }
+  if (epi.mode == GEMM_GEGLU) {
+    const uint32_t o0 = pack_bf16x2(v[0] * gelu_erf(v[1]), v[2] * gelu_erf(v[3]));
+    const uint32_t o1 = pack_bf16x2(v[4] * gelu_erf(v[5]), v[6] * gelu_erf(v[7]));
+    *reinterpret_cast<uint2*>(epi.out + (size_t)row * epi.ld_out + c / 2) = make_uint2(o0, o1);
+    return;
+  }
+  if (epi.residual) {
+    const uint4 r = *reinterpret_cast<const uint4*>(epi.residual + (size_t)row * epi.ld_res + c);
+    v[0] += bf16lo(r.x); v[1] += bf16hi(r.x); v[2] += bf16lo(r.y); v[3] += bf16hi(r.y);
+    v[4] += bf16lo(r.z); v[5] += bf16hi(r.z); v[6] += bf16lo(r.w); v[7] += bf16hi(r.w);
+  }
+  if (epi.f16_begin > 0 && c >= epi.f16_begin) {
+    *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) =
+        make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
+    return;
+  }
+  const uint4 o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                             pack_bf16x2(v[6], v[7]));
+  *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) = o;
+  const uint32_t w[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float lo = bf16lo(w[j]), hi = bf16hi(w[j]);
+    rs1 += lo + hi;
+    rs2 = fmaf(lo, lo, fmaf(hi, hi, rs2));
+  }
+}
+
 // Split-K reduction: out = epilogue(sum over splits of partial), 8 columns per
-// thread, splits added in index order (deterministic).
+// thread. With row statistics requested, each warp takes one 256-column segment
+// of one row and adds its shuffle-reduced sums into the row's fixed-point pair.
 __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N, GemmEpi epi) {
   pdl_wait();
   pdl_trigger();
   const int V = N / 8;
-  const size_t total = (size_t)M * V;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-    const int row = (int)(i / V);
-    const int c = (int)(i % V) * 8;
-    float v[8];
-    const float4* p0 = reinterpret_cast<const float4*>(partial + (size_t)row * N + c);
-    float4 a = p0[0], b = p0[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    for (int z = 1; z < splits; ++z) {
-      const float4* pz = reinterpret_cast<const float4*>(partial + ((size_t)z * M + row) * N + c);
-      a = pz[0];
-      b = pz[1];
-      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w; v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  if (!epi.rowstat_out) {
+    const size_t total = (size_t)M * V;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+      float r1 = 0.f, r2 = 0.f;
+      splitk_reduce_vec(partial, splits, M, N, epi, (int)(i / V), (int)(i % V) * 8, r1, r2);
     }
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int segs = (V + 31) / 32;
+  const size_t warps = (size_t)M * segs;
+  const size_t nwarps = (size_t)gridDim.x * (blockDim.x >> 5);
+  for (size_t wi = blockIdx.x * (size_t)(blockDim.x >> 5) + (threadIdx.x >> 5); wi < warps; wi += nwarps) {
+    const int row = (int)(wi / segs);
+    const int vec = (int)(wi % segs) * 32 + lane;
+    float r1 = 0.f, r2 = 0.f;
+    if (vec < V) splitk_reduce_vec(partial, splits, M, N, epi, row, vec * 8, r1, r2);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float add = 0.f;
-      if (epi.bias) add += __bfloat162float(epi.bias[c + j]);
-      if (epi.bias2) add += __bfloat162float(epi.bias2[c + j]);
-      if (epi.colvec) add += epi.colvec[c + j];
-      v[j] += add;
+    for (int o = 16; o; o >>= 1) {
+      r1 += __shfl_xor_sync(0xffffffffu, r1, o);
+      r2 += __shfl_xor_sync(0xffffffffu, r2, o);
     }
-    if (epi.mode == GEMM_GEGLU) {
-      const uint32_t o0 = pack_bf16x2(v[0] * gelu_erf(v[1]), v[2] * gelu_erf(v[3]));
-      const uint32_t o1 = pack_bf16x2(v[4] * gelu_erf(v[5]), v[6] * gelu_erf(v[7]));
-      *reinterpret_cast<uint2*>(epi.out + (size_t)row * epi.ld_out + c / 2) = make_uint2(o0, o1);
-      continue;
+    if (lane == 0) {
+      atomicAdd(epi.rowstat_out + 2 * row, (unsigned long long)llrint((double)r1 * kRowSumScale));
+      atomicAdd(epi.rowstat_out + 2 * row + 1, (unsigned long long)llrint((double)r2 * kRowSqScale));
     }
-    if (epi.residual) {
-      const uint4 r = *reinterpret_cast<const uint4*>(epi.residual + (size_t)row * epi.ld_res + c);
-      v[0] += bf16lo(r.x); v[1] += bf16hi(r.x); v[2] += bf16lo(r.y); v[3] += bf16hi(r.y);
-      v[4] += bf16lo(r.z); v[5] += bf16hi(r.z); v[6] += bf16lo(r.w); v[7] += bf16hi(r.w);
-    }
-    if (epi.f16_begin > 0 && c >= epi.f16_begin)
-      *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) =
-          make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
-    else
-      *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) =
-          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
   }
 }
 

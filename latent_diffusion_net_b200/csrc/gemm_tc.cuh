@@ -48,7 +48,27 @@ struct GemmEpi {
   int32_t ld_out;
   int32_t mode;                   // GemmMode
   int32_t f16_begin;              // > 0: output columns >= f16_begin are stored as FP16 (a multiple of 32)
+  // Row statistics for a LayerNorm folded into the next GEMM. rowstat_out: each
+  // output row's sum and sum of squares of the stored BF16 values are added into
+  // rowstat_out[2*row .. 2*row+1] as 64-bit fixed point (scales 2^24 and 2^18);
+  // the buffer must be zero before the launch. rowstat_in: the A operand is the
+  // raw (not normalised) input x whose row sums are there; the epilogue then
+  // forms rstd*(acc - mean*colscale[n]) + colvec[n] with mean and rstd over
+  // ln_cols values and ln_eps (a LayerNorm with gamma folded into B, colscale =
+  // row sums of that B, colvec = B times beta plus bias).
+  unsigned long long* rowstat_out;
+  const unsigned long long* rowstat_in;
+  // Zeroed by this launch once every earlier kernel on the stream has finished
+  // (the other row-statistics buffer, whose last reader ran before).
+  unsigned long long* rowstat_clear;
+  int64_t rowstat_clear_elems;
+  const float* colscale;
+  int32_t ln_cols;
+  float ln_eps;
 };
+
+constexpr double kRowSumScale = 16777216.0;  // 2^24
+constexpr double kRowSqScale = 262144.0;     // 2^18
 
 // A full problem: output grid Ho x Wo (M = Ho*Wo rows), N output features.
 // When the tile grid cannot fill the GPU and an FP32 split-K buffer is given,

@@ -13,9 +13,6 @@ namespace sdk {
 int launch_groupnorm(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G, float eps,
                      const __nv_bfloat16* gamma, const __nv_bfloat16* beta, int silu, __nv_bfloat16* y,
                      unsigned long long* acc, int num_sms, cudaStream_t st);
-int launch_layernorm(const __nv_bfloat16* x, int N, int C, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,
-                     float eps, __nv_bfloat16* y, cudaStream_t st);
-
 // Time embedding: phi(t) sinusoid [proj_dim] into out (FP32).
 int launch_sinusoid(float t, int proj_dim, float* out, cudaStream_t st);
 

@@ -7,8 +7,8 @@
 // of the up path) and is never materialised: a vector of 8 channels is read
 // from whichever source holds it.
 //
-// LayerNorm (BasicTransformer Block bullet of the tutorial page): per token
-// over C, biased variance, then scale/shift.
+// The transformer's LayerNorms are folded into the GEMMs they feed (gemm_tc.cu
+// row statistics), so no LayerNorm kernel exists.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -156,74 +156,6 @@ __global__ void gn_apply_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
   }
 }
 
-// ------------------------------------------------------------------ LayerNorm
-// T lanes per token (T = 4..32, a power of two), each lane holding at most 8
-// 16-byte vectors of the row in registers; two-pass mean/variance.
-constexpr int kLnMaxVec = 8;
-
-__global__ void ln_kernel(const __nv_bfloat16* __restrict__ x, int N, int C, int T,
-                          const __nv_bfloat16* __restrict__ gamma, const __nv_bfloat16* __restrict__ beta, float eps,
-                          __nv_bfloat16* __restrict__ y) {
-  pdl_wait();
-  pdl_trigger();
-  const int gtid = blockIdx.x * blockDim.x + threadIdx.x;
-  const int tok = gtid / T;
-  const int sub = gtid % T;
-  const bool active = tok < N;
-  const int V = C >> 3;
-  const __nv_bfloat16* row = x + (size_t)(active ? tok : 0) * C;
-  uint4 buf[kLnMaxVec];
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < kLnMaxVec; ++i) {
-    const int v = sub + T * i;
-    if (active && v < V) {
-      buf[i] = *reinterpret_cast<const uint4*>(row + v * 8);
-      s += bf16lo(buf[i].x) + bf16hi(buf[i].x) + bf16lo(buf[i].y) + bf16hi(buf[i].y) + bf16lo(buf[i].z) +
-           bf16hi(buf[i].z) + bf16lo(buf[i].w) + bf16hi(buf[i].w);
-    }
-  }
-  for (int o = T >> 1; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  const float mean = s / C;
-  float q = 0.f;
-#pragma unroll
-  for (int i = 0; i < kLnMaxVec; ++i) {
-    const int v = sub + T * i;
-    if (active && v < V) {
-      const float f[8] = {bf16lo(buf[i].x), bf16hi(buf[i].x), bf16lo(buf[i].y), bf16hi(buf[i].y),
-                          bf16lo(buf[i].z), bf16hi(buf[i].z), bf16lo(buf[i].w), bf16hi(buf[i].w)};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) q = fmaf(f[j] - mean, f[j] - mean, q);
-    }
-  }
-  for (int o = T >> 1; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-  const float rstd = rsqrtf(q / C + eps);
-  if (!active) return;
-  __nv_bfloat16* out = y + (size_t)tok * C;
-#pragma unroll
-  for (int i = 0; i < kLnMaxVec; ++i) {
-    const int v = sub + T * i;
-    if (v < V) {
-      const int c = v * 8;
-      const uint4 gw = __ldg(reinterpret_cast<const uint4*>(gamma + c));
-      const uint4 bw = __ldg(reinterpret_cast<const uint4*>(beta + c));
-      const float f[8] = {bf16lo(buf[i].x), bf16hi(buf[i].x), bf16lo(buf[i].y), bf16hi(buf[i].y),
-                          bf16lo(buf[i].z), bf16hi(buf[i].z), bf16lo(buf[i].w), bf16hi(buf[i].w)};
-      const float g[8] = {bf16lo(gw.x), bf16hi(gw.x), bf16lo(gw.y), bf16hi(gw.y),
-                          bf16lo(gw.z), bf16hi(gw.z), bf16lo(gw.w), bf16hi(gw.w)};
-      const float b[8] = {bf16lo(bw.x), bf16hi(bw.x), bf16lo(bw.y), bf16hi(bw.y),
-                          bf16lo(bw.z), bf16hi(bw.z), bf16lo(bw.w), bf16hi(bw.w)};
-      float o[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = fmaf((f[j] - mean) * rstd, g[j], b[j]);
-      *reinterpret_cast<uint4*>(out + c) =
-          make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
-    }
-  }
-}
-
-// ------------------------------------------------------------------ launchers
-
 int launch_groupnorm(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G, float eps,
                      const __nv_bfloat16* gamma, const __nv_bfloat16* beta, int silu, __nv_bfloat16* y,
                      unsigned long long* acc, int num_sms, cudaStream_t st) {
@@ -243,18 +175,6 @@ int launch_groupnorm(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, i
   if (blocks > 2 * num_sms) blocks = 2 * num_sms;
   return (int)launch_pdl(gn_apply_kernel, dim3(blocks), dim3(256), C * sizeof(float2), st, x0, C0, x1, C1, HW, G, eps,
                          (const unsigned long long*)acc, gamma, beta, silu, y);
-}
-
-int launch_layernorm(const __nv_bfloat16* x, int N, int C, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,
-                     float eps, __nv_bfloat16* y, cudaStream_t st) {
-  const int V = C / 8;
-  int T = 4;
-  while (T < 32 && (V + T - 1) / T > kLnMaxVec) T <<= 1;
-  if ((V + T - 1) / T > kLnMaxVec) return -1;
-  const int threads = 256;
-  const long total = (long)N * T;
-  const int blocks = (int)((total + threads - 1) / threads);
-  return (int)launch_pdl(ln_kernel, dim3(blocks), dim3(threads), 0, st, x, N, C, T, gamma, beta, eps, y);
 }
 
 }  // namespace sdk

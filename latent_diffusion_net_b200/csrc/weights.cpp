@@ -30,6 +30,15 @@ int64_t Table::add(const std::string& name, std::initializer_list<int64_t> shape
   return x.packed_off;
 }
 
+int64_t Table::add_derived(const Derived& x0) {
+  Derived x = x0;
+  packed_bytes = (packed_bytes + 255) & ~int64_t(255);
+  x.out_off = packed_bytes;
+  packed_bytes += x.rows * 4;
+  d.push_back(x);
+  return x.out_off;
+}
+
 TimeW add_time(Table& tab, const std::string& p, int proj, int temb) {
   TimeW w;
   w.l1w = tab.add(p + ".lin1.weight", {temb, proj}, SD_KIND_WEIGHT, proj);
@@ -99,27 +108,44 @@ TxW add_transformer(Table& tab, const std::string& p, int C, int depth, int D) {
     const std::string b = p + ".blocks." + std::to_string(d);
     TxBlockW k;
     k.ln1g = tab.add(b + ".ln1.gamma", {C}, SD_KIND_NORM_GAMMA, 0);
+    const int ln1g = tab.last();
     k.ln1b = tab.add(b + ".ln1.beta", {C}, SD_KIND_NORM_BETA, 0);
-    // q, k, v are consecutive (each a multiple of 256 bytes): one [3C, C] matrix
-    k.qkv = tab.add(b + ".attn1.q.weight", {C, C}, SD_KIND_WEIGHT, C);
-    tab.add(b + ".attn1.k.weight", {C, C}, SD_KIND_WEIGHT, C);
-    tab.add(b + ".attn1.v.weight", {C, C}, SD_KIND_WEIGHT, C);
+    const int ln1b = tab.last();
+    // q, k, v are consecutive (each a multiple of 256 bytes): one [3C, C] matrix, packed with LN1's gamma
+    k.qkv = tab.add(b + ".attn1.q.weight", {C, C}, SD_KIND_WEIGHT, C, PACK_LNFOLD, ln1g);
+    const int qkv = tab.last();
+    tab.add(b + ".attn1.k.weight", {C, C}, SD_KIND_WEIGHT, C, PACK_LNFOLD, ln1g);
+    tab.add(b + ".attn1.v.weight", {C, C}, SD_KIND_WEIGHT, C, PACK_LNFOLD, ln1g);
     k.o1w = tab.add(b + ".attn1.out.weight", {C, C}, SD_KIND_WEIGHT, C);
     k.o1b = tab.add(b + ".attn1.out.bias", {C}, SD_KIND_BIAS, C);
     k.ln2g = tab.add(b + ".ln2.gamma", {C}, SD_KIND_NORM_GAMMA, 0);
+    const int ln2g = tab.last();
     k.ln2b = tab.add(b + ".ln2.beta", {C}, SD_KIND_NORM_BETA, 0);
-    k.q2 = tab.add(b + ".attn2.q.weight", {C, C}, SD_KIND_WEIGHT, C);
+    const int ln2b = tab.last();
+    k.q2 = tab.add(b + ".attn2.q.weight", {C, C}, SD_KIND_WEIGHT, C, PACK_LNFOLD, ln2g);
+    const int q2 = tab.last();
     // k, v of the cross-attention are consecutive: one [2C, D] matrix
     k.kv2 = tab.add(b + ".attn2.k.weight", {C, D}, SD_KIND_WEIGHT, D);
     tab.add(b + ".attn2.v.weight", {C, D}, SD_KIND_WEIGHT, D);
     k.o2w = tab.add(b + ".attn2.out.weight", {C, C}, SD_KIND_WEIGHT, C);
     k.o2b = tab.add(b + ".attn2.out.bias", {C}, SD_KIND_BIAS, C);
     k.ln3g = tab.add(b + ".ln3.gamma", {C}, SD_KIND_NORM_GAMMA, 0);
+    const int ln3g = tab.last();
     k.ln3b = tab.add(b + ".ln3.beta", {C}, SD_KIND_NORM_BETA, 0);
-    k.f1w = tab.add(b + ".ff.w1.weight", {8 * C, C}, SD_KIND_WEIGHT, C, PACK_GEGLU_ROWS);
+    const int ln3b = tab.last();
+    k.f1w = tab.add(b + ".ff.w1.weight", {8 * C, C}, SD_KIND_WEIGHT, C, PACK_LNFOLD_GEGLU, ln3g);
+    const int f1w = tab.last();
     k.f1b = tab.add(b + ".ff.w1.bias", {8 * C}, SD_KIND_BIAS, C, PACK_GEGLU_BIAS);
+    const int f1b = tab.last();
     k.f2w = tab.add(b + ".ff.w2.weight", {C, 4 * C}, SD_KIND_WEIGHT, 4 * C);
     k.f2b = tab.add(b + ".ff.w2.bias", {C}, SD_KIND_BIAS, 4 * C);
+    // column terms of the three folded LayerNorms, after the canonical tensors of this block
+    k.qkv_c1 = tab.add_derived({false, 0, 3 * C, C, qkv, -1, -1, false});
+    k.qkv_c2 = tab.add_derived({true, 0, 3 * C, C, qkv, ln1b, -1, false});
+    k.q2_c1 = tab.add_derived({false, 0, C, C, q2, -1, -1, false});
+    k.q2_c2 = tab.add_derived({true, 0, C, C, q2, ln2b, -1, false});
+    k.f1_c1 = tab.add_derived({false, 0, 8 * C, C, f1w, -1, -1, true});
+    k.f1_c2 = tab.add_derived({true, 0, 8 * C, C, f1w, ln3b, f1b, true});
     w.blocks.push_back(k);
   }
   w.pow_ = tab.add(p + ".proj_out.weight", {C, C}, SD_KIND_WEIGHT, C);
@@ -178,6 +204,31 @@ UNetW add_unet(Table& tab, const sd_unet_cfg& cfg) {
   return u;
 }
 
+namespace {
+
+float bf16_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+// Round to nearest even; inputs here are finite products of two BF16 values.
+uint16_t f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+// Canonical row of packed row r of a (possibly GEGLU-interleaved) [rows][K] matrix.
+int64_t canon_row(int64_t r, int64_t rows, bool geglu) {
+  if (!geglu) return r;
+  return (r & 1) ? rows / 2 + (r >> 1) : (r >> 1);
+}
+
+}  // namespace
+
 void pack(const Table& tab, const uint16_t* canon, uint8_t* packed) {
   memset(packed, 0, (size_t)tab.packed_bytes);
   for (const Tensor& x : tab.t) {
@@ -219,6 +270,40 @@ void pack(const Table& tab, const uint16_t* canon, uint8_t* packed) {
           dst[2 * j + 1] = src[half + j];
         }
         break;
+      }
+      case PACK_LNFOLD:
+      case PACK_LNFOLD_GEGLU: {
+        const uint16_t* gamma = canon + tab.t[x.aux].canon_off;
+        const int64_t R = x.shape[0], K = x.shape[1];
+        const bool geglu = x.pack == PACK_LNFOLD_GEGLU;
+        for (int64_t r = 0; r < R; ++r) {
+          const uint16_t* row = src + canon_row(r, R, geglu) * K;
+          for (int64_t k = 0; k < K; ++k) dst[r * K + k] = f32_to_bf16(bf16_to_f32(row[k]) * bf16_to_f32(gamma[k]));
+        }
+        break;
+      }
+    }
+  }
+  // derived column terms (after every tensor: c1 reads the packed W')
+  for (const Derived& x : tab.d) {
+    float* out = reinterpret_cast<float*>(packed + x.out_off);
+    const Tensor& wt = tab.t[x.w_tensor];
+    if (!x.c2) {
+      const uint16_t* wp = reinterpret_cast<const uint16_t*>(packed + wt.packed_off);
+      for (int64_t r = 0; r < x.rows; ++r) {
+        double s = 0;
+        for (int64_t k = 0; k < x.K; ++k) s += bf16_to_f32(wp[r * x.K + k]);
+        out[r] = (float)s;
+      }
+    } else {
+      const uint16_t* wc = canon + wt.canon_off;
+      const uint16_t* beta = canon + tab.t[x.beta_tensor].canon_off;
+      const uint16_t* bias = x.bias_tensor >= 0 ? canon + tab.t[x.bias_tensor].canon_off : nullptr;
+      for (int64_t r = 0; r < x.rows; ++r) {
+        const int64_t cr = canon_row(r, x.rows, x.geglu);
+        double s = bias ? bf16_to_f32(bias[cr]) : 0.0;
+        for (int64_t k = 0; k < x.K; ++k) s += (double)bf16_to_f32(wc[cr * x.K + k]) * bf16_to_f32(beta[k]);
+        out[r] = (float)s;
       }
     }
   }

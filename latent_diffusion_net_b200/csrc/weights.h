@@ -16,7 +16,22 @@ enum Pack : int {
   PACK_CONV_KRSC,    // [O][C][kh][kw] -> [O][kh][kw][C]
   PACK_CONV_IM2COL,  // [O][C][3][3]  -> [O][Kp], k = (ky*3+kx)*C + c, zero-padded to Kp
   PACK_GEGLU_ROWS,   // [8C][C]: row 2j = value row j, row 2j+1 = gate row 4C + j
-  PACK_GEGLU_BIAS    // [8C]: same interleave
+  PACK_GEGLU_BIAS,   // [8C]: same interleave
+  PACK_LNFOLD,       // [R][K] times the LayerNorm gamma of tensor `aux` along K, rounded to BF16
+  PACK_LNFOLD_GEGLU  // PACK_GEGLU_ROWS of the PACK_LNFOLD product
+};
+
+// FP32 vectors derived from several canonical tensors (packed after them): for
+// a linear layer fed by a LayerNorm, with W' = W * gamma (as packed),
+// c1[r] = sum_k W'[r][k] and c2[r] = sum_k W[r][k] * beta[k] + bias[r].
+struct Derived {
+  bool c2;          // false: c1 from the packed W'; true: c2 from canonical W, beta, bias
+  int64_t out_off;  // packed byte offset of the FP32 vector
+  int64_t rows, K;
+  int w_tensor;     // first canonical tensor of the rows (consecutive tensors continue them)
+  int beta_tensor;  // c2: LayerNorm beta
+  int bias_tensor;  // c2: bias or -1
+  bool geglu;       // rows interleaved as PACK_GEGLU_ROWS
 };
 
 struct Tensor {
@@ -39,11 +54,15 @@ struct Tensor {
 
 struct Table {
   std::vector<Tensor> t;
+  std::vector<Derived> d;
   int64_t canon_elems = 0;
   int64_t packed_bytes = 0;
   // Appends a tensor; returns its packed byte offset.
   int64_t add(const std::string& name, std::initializer_list<int64_t> shape, int kind, int fan_in,
               int pack = PACK_COPY, int aux = 0);
+  // Appends a derived FP32 vector of `rows` entries; returns its packed byte offset.
+  int64_t add_derived(const Derived& x);
+  int last() const { return (int)t.size() - 1; }
 };
 
 // Packed byte offsets of each module's tensors.
@@ -62,6 +81,9 @@ struct ResW {
 };
 struct TxBlockW {
   int64_t ln1g, ln1b, qkv, o1w, o1b, ln2g, ln2b, q2, kv2, o2w, o2b, ln3g, ln3b, f1w, f1b, f2w, f2b;
+  // LayerNorm folded into the following linear: qkv, q2 and f1w are packed as
+  // W * gamma; c1 / c2 are the FP32 column terms of the GEMM epilogue
+  int64_t qkv_c1, qkv_c2, q2_c1, q2_c2, f1_c1, f1_c2;
 };
 struct TxW {
   int C, depth, ctx_dim;

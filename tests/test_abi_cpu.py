@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 
 from latent_diffusion_net_b200 import binding as B
+from latent_diffusion_net_b200 import synth
 from oracle import model
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -92,16 +93,20 @@ def test_pack_conv_krsc_and_geglu_interleave():
     src = canon[r["canon_offset"]:r["canon_offset"] + O * Ci * 9].reshape(O, Ci, 3, 3)
     dst = packed[r["packed_offset"] // 2:r["packed_offset"] // 2 + O * Ci * 9].reshape(O, 3, 3, Ci)
     np.testing.assert_array_equal(dst, src.transpose(0, 2, 3, 1))
+    # FF1 rows: value/gate interleave of W * gamma(LN3), rounded to BF16 (the LayerNorm fold)
     tcfg = B.transformer_cfg(4, 4, 256, 1, ctx_dim=256)
     rows, canon_n, packed_n = B.sd_transformer_weight_layout(tcfg)
-    canon = (np.arange(canon_n, dtype=np.int64) % 65521).astype(np.uint16)
+    canon = synth.normal_bf16_bits(99, 0, canon_n)
     packed = B.sd_transformer_pack_weights(tcfg, canon, packed_n).view(np.uint16)
     r = [x for x in rows if x["name"].endswith("ff.w1.weight")][0]
+    g = [x for x in rows if x["name"].endswith("ln3.gamma")][0]
     R, K = r["shape"]
-    src = canon[r["canon_offset"]:r["canon_offset"] + R * K].reshape(R, K)
+    src = synth.bf16_bits_to_f32(canon[r["canon_offset"]:r["canon_offset"] + R * K]).reshape(R, K)
+    gamma = synth.bf16_bits_to_f32(canon[g["canon_offset"]:g["canon_offset"] + K])
+    folded = synth.f32_to_bf16_bits((src * gamma[None, :]).astype(np.float32))
     dst = packed[r["packed_offset"] // 2:r["packed_offset"] // 2 + R * K].reshape(R, K)
-    np.testing.assert_array_equal(dst[0::2], src[:R // 2])
-    np.testing.assert_array_equal(dst[1::2], src[R // 2:])
+    np.testing.assert_array_equal(dst[0::2], folded[:R // 2])
+    np.testing.assert_array_equal(dst[1::2], folded[R // 2:])
     # q, k, v contiguous: [3C, C]
     q = [x for x in rows if x["name"].endswith("attn1.q.weight")][0]
     v = [x for x in rows if x["name"].endswith("attn1.v.weight")][0]
