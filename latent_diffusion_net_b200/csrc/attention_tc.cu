@@ -326,16 +326,24 @@ __global__ void __launch_bounds__(192, 2)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(s_free);
-      float mx = -INFINITY;
-      if (kvalid >= kAK) {
+      // row maximum over four independent chains (a single chain of 128 dependent
+      // maxima would cost its full latency per tile)
+      float mx;
+      {
+        if (kvalid < kAK) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          if (i >= kvalid) sv[i] = __float_as_uint(-INFINITY);
-          mx = fmaxf(mx, __uint_as_float(sv[i]));
+          for (int i = 0; i < 128; ++i)
+            if (i >= kvalid) sv[i] = __float_as_uint(-INFINITY);
         }
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; i += 4) {
+          m0 = fmaxf(m0, __uint_as_float(sv[i]));
+          m1 = fmaxf(m1, __uint_as_float(sv[i + 1]));
+          m2 = fmaxf(m2, __uint_as_float(sv[i + 2]));
+          m3 = fmaxf(m3, __uint_as_float(sv[i + 3]));
+        }
+        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
       }
       // the previous PV product must be done before P is overwritten or O rescaled
       if (t > 0 && !mbar_wait(pv_done, (t - 1) & 1, abort_flag, args.err)) break;
@@ -362,6 +370,8 @@ __global__ void __launch_bounds__(192, 2)
         }
       }
       // P = exp2(s*scale*log2e - m_used) in BF16 (masked keys give exp2(-inf) = 0), row sum
+      // accumulated in two independent chains per tile
+      float la = 0.f, lb = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -369,7 +379,8 @@ __global__ void __launch_bounds__(192, 2)
         for (int i = 0; i < 16; ++i) {
           const float p0 = ex2(fmaf(__uint_as_float(sv[c * 32 + 2 * i]), sl2, -m_used));
           const float p1 = ex2(fmaf(__uint_as_float(sv[c * 32 + 2 * i + 1]), sl2, -m_used));
-          l += p0 + p1;
+          la += p0;
+          lb += p1;
           pk[i] = pack_bf16x2_alu(p0, p1);
         }
         // keys c*32 .. c*32+31 = half c/2, 16-byte chunks 4*(c&1) .. +3, swizzled by row
@@ -382,6 +393,7 @@ __global__ void __launch_bounds__(192, 2)
                        : "memory");
         }
       }
+      l += la + lb;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
