@@ -20,12 +20,18 @@ Topology sources (page title, section):
   Transformer bullets (GroupNorm + Linear/Conv + BasicTransformer Blocks +
   Linear/Conv, with the block input added back); DownSample and UpSample bullets.
 
-Readings where the pages are silent (each is listed in the design doc): GroupNorm and
-LayerNorm eps 1e-5, 32 groups, biased variance; Q/K/V projections without bias,
-out-projection / proj_in / proj_out / FF with bias; head_dim 64; no attention
-mask; GEGLU value half first, exact-erf GELU; the 12-entry skip stack popped
-last-in-first-out with concatenation order [h, skip]; symmetric padding 1 for the
-stride-2 convolution.
+Readings where the pages are silent (each is listed with the design notes):
+GroupNorm and LayerNorm eps 1e-5, 32 groups, biased variance; Q/K/V projections
+without bias, out-projection / proj_in / proj_out / FF with bias; head_dim 64;
+no attention mask; GEGLU value half first, exact-erf GELU; the 12-entry skip
+stack popped last-in-first-out with concatenation order [h, skip]; symmetric
+padding 1 for the stride-2 convolution.
+
+Parity unpinned: the absolute output values of ``resblock``, ``transformer``
+and ``unet_step``. No page prints a numeric output of a block or of the step,
+so these compositions are pinned only through their parts (every op in
+``ops`` is pinned), identities (zeroed sublayers reduce a block to a known
+function), the pages' shapes and parameter totals.
 """
 from __future__ import annotations
 
