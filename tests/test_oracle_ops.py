@@ -204,6 +204,29 @@ def attention_brute(q, k, v, hd):
     return out
 
 
+def test_layer_norm_folds_into_the_following_linear():
+    """The identity the GPU path uses instead of a LayerNorm kernel:
+    LN(x) W^T + b = rstd (x (W*gamma)^T - mean c1) + c2, c1 = rowsum(W*gamma),
+    c2 = W beta + b, with mean and rstd of each row of x (biased variance) and
+    the row statistics taken from sum x and sum x^2 as the GPU accumulates them."""
+    rng = np.random.default_rng(7)
+    N, C, O, eps = 11, 48, 20, 1e-5
+    x = rng.normal(0.3, 1.7, (N, C))
+    gamma, beta = 1 + 0.2 * rng.normal(size=C), 0.3 * rng.normal(size=C)
+    W, bias = rng.normal(size=(O, C)) / math.sqrt(C), rng.normal(size=O)
+    ref = ops.linear(ops.layer_norm(x, gamma, beta, eps), W, bias)
+    Wg = W * gamma[None, :]
+    c1, c2 = Wg.sum(axis=1), W @ beta + bias
+    s1, s2 = x.sum(axis=1), (x * x).sum(axis=1)
+    mean = s1 / C
+    rstd = 1 / np.sqrt(s2 / C - mean ** 2 + eps)
+    folded = rstd[:, None] * (x @ Wg.T - mean[:, None] * c1[None, :]) + c2[None, :]
+    np.testing.assert_allclose(folded, ref, rtol=1e-11, atol=1e-11)
+    # a dropped term is caught: without c1 (or with gamma left out) the results differ
+    assert not np.allclose(rstd[:, None] * (x @ Wg.T) + c2[None, :], ref, atol=1e-3)
+    assert not np.allclose(rstd[:, None] * (x @ W.T - mean[:, None] * W.sum(axis=1)) + c2[None, :], ref, atol=1e-3)
+
+
 def test_attention_brute_force_small():
     r = rng(10)
     q, k, v = (r.standard_normal((5, 8)) for _ in range(3))
