@@ -345,51 +345,58 @@ __global__ void __launch_bounds__(192, 2)
         }
         mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
       }
-      // the previous PV product must be done before P is overwritten or O rescaled
-      if (t > 0 && !mbar_wait(pv_done, (t - 1) & 1, abort_flag, args.err)) break;
-      tc_fence_after();
+      // new running maximum; O is rescaled (after the wait below) only when it grew by more than 2^8
+      float alpha = 1.f;
+      bool rescale = false;
       if (first) {
         m_used = mx * sl2;
         l = 0.f;
       } else {
         const float m_new = fmaxf(m_used, mx * sl2);
         if (m_new > m_used + 8.f) {
-          const float alpha = ex2(m_used - m_new);
+          alpha = ex2(m_used - m_new);
           l *= alpha;
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(tOrow + c * 32, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st_32x32b_x32(tOrow + c * 32, r);
-          }
-          tmem_st_wait();
           m_used = m_new;
+          rescale = true;
         }
       }
-      // P = exp2(s*scale*log2e - m_used) in BF16 (masked keys give exp2(-inf) = 0), row sum
-      // accumulated in two independent chains per tile
+      // P = exp2(s*scale*log2e - m_used) as packed BF16 pairs in registers (masked keys give
+      // exp2(-inf) = 0) while the previous PV product may still be running; row sum in two chains
+      uint32_t pk[64];
       float la = 0.f, lb = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2(fmaf(__uint_as_float(sv[2 * i]), sl2, -m_used));
+        const float p1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -m_used));
+        la += p0;
+        lb += p1;
+        pk[i] = pack_bf16x2_alu(p0, p1);
+      }
+      // the previous PV product must be done before P is overwritten or O rescaled
+      if (t > 0 && !mbar_wait(pv_done, (t - 1) & 1, abort_flag, args.err)) break;
+      tc_fence_after();
+      if (rescale) {
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tOrow + c * 32, r);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(sv[c * 32 + 2 * i]), sl2, -m_used));
-          const float p1 = ex2(fmaf(__uint_as_float(sv[c * 32 + 2 * i + 1]), sl2, -m_used));
-          la += p0;
-          lb += p1;
-          pk[i] = pack_bf16x2_alu(p0, p1);
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st_32x32b_x32(tOrow + c * 32, r);
         }
+        tmem_st_wait();
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
         // keys c*32 .. c*32+31 = half c/2, 16-byte chunks 4*(c&1) .. +3, swizzled by row
         const uint32_t hrow = prow0 + (c >> 1) * kTileBytes;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int chunk = ((c & 1) * 4 + q) ^ (row & 7);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(hrow + chunk * 16), "r"(pk[4 * q]),
-                       "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+          const int k = c * 16 + 4 * q;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(hrow + chunk * 16), "r"(pk[k]),
+                       "r"(pk[k + 1]), "r"(pk[k + 2]), "r"(pk[k + 3])
                        : "memory");
         }
       }
