@@ -269,7 +269,8 @@ sd_status sd_query_device_status(void* workspace, sd_stream_t stream);
  * them. sd_profile_read() returns the records of the last recording with their
  * elapsed times (ms < 0 where the events have not completed). */
 typedef struct {
-  char kernel[24];  /* "gemm_tc", "attention", "gn_stats", "gn_apply", "layernorm", "gemv", ... */
+  char kernel[24];  /* "gemm_tc", "attention", "groupnorm", "gemv", ... (SD_FAMILY_LAYERNORM is unused:
+                       the LayerNorms are folded into the GEMMs) */
   int32_t family;   /* SD_FAMILY_* */
   int32_t kernels;  /* kernels enqueued by this launch (a split-K GEMM enqueues 2) */
   double flops;

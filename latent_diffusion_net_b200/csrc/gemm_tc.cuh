@@ -71,9 +71,10 @@ constexpr double kRowSumScale = 16777216.0;  // 2^24
 constexpr double kRowSqScale = 262144.0;     // 2^18
 
 // A full problem: output grid Ho x Wo (M = Ho*Wo rows), N output features.
-// When the tile grid cannot fill the GPU and an FP32 split-K buffer is given,
-// the reduction is split over blockIdx.z and a second kernel adds the partial
-// products in a fixed order and applies the epilogue.
+// When its cost model says it pays and an FP32 split-K buffer is given, the
+// planner splits the reduction into K ranges (separate work units of the
+// persistent kernel) and a second kernel adds the partial products in a fixed
+// order and applies the epilogue.
 struct GemmProblem {
   int32_t Ho, Wo, N;
   int32_t na, nb, nseg;

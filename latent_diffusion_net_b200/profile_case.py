@@ -7,7 +7,7 @@ seeded [hw, hw, C] input; ``transformer`` runs a Transformer2DModel (depth 1,
 block's entry point, so a kernel capture with ``-k`` and ``-c`` selects
 launches by their order inside the block (the ResnetBlock2D issues GroupNorm,
 conv1, GroupNorm, conv2; the Transformer2DModel issues its GroupNorm, the
-proj_in GEMM, LayerNorm, the QKV GEMM, self-attention, ...). Prints the mean
+proj_in GEMM, the QKV GEMM with LayerNorm folded in, self-attention, ...). Prints the mean
 time per call measured with CUDA events after the warm-up calls.
 """
 from __future__ import annotations

@@ -60,3 +60,22 @@ def test_reference_arm_other_ranks_exit_without_work():
         steps, warmup = 1, 0
 
     assert bench.run_reference(Args, rank=1, world=2) == 0
+
+
+def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch):
+    """bench.py reports the committed DRAM traffic of a kernel only while the
+    kernel's source is byte-identical to the one the capture was taken on."""
+    import hashlib
+
+    src = tmp_path / "kernel.cu"
+    src.write_text("// version 1\n")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    digest = hashlib.sha256(src.read_bytes()).hexdigest()
+    (prof / "k_dram_traffic_unet_step_sd21_96.md").write_text(
+        "summary\n\ntraffic_bytes_per_launch: 1234\nsource: kernel.cu\nsource_sha256: " + digest + "\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("k") == 1234.0
+    src.write_text("// version 2\n")
+    assert bench.measured_traffic("k") is None
+    assert bench.measured_traffic("missing") is None
