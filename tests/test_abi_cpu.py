@@ -162,6 +162,14 @@ def test_host_validation_without_gpu():
     assert B.sd_unet_step(u, fake, fake, 500.0, fake, fake, fake, 10 ** 10, check=False) == 3
     d = B.conv_cfg(9, 8, 320, 320)
     assert B.sd_conv_fwd(d, B.SD_CONV_DOWNSAMPLE, fake, fake, None, None, fake, fake, 10 ** 9, check=False) == 2
+    # empty images are rejected as bad shapes before anything is launched
+    assert B.sd_resblock_fwd(B.resblock_cfg(0, 8, 320, 320), fake, fake, None, fake, fake, fake, 10 ** 9,
+                             check=False) == 2
+    assert B.sd_transformer_fwd(B.transformer_cfg(8, 0, 320), fake, fake, fake, fake, fake, 10 ** 9, check=False) == 2
+    assert B.sd_conv_fwd(B.conv_cfg(0, 8, 320, 320), B.SD_CONV_UPSAMPLE, fake, fake, None, None, fake, fake, 10 ** 9,
+                         check=False) == 2
+    assert B.sd_unet_step(B.unet_cfg(height=0, width=96), fake, fake, 500.0, fake, fake, fake, 10 ** 10,
+                          check=False) == 2
     # a well-formed call on a machine without a usable B200 fails cleanly, never crashes
     s = B.sd_resblock_fwd(cfg, fake, fake, None, fake, fake, fake, ws, check=False)
     assert s in (0, 6, 7) and (s != 0 or os.environ.get("CUDA_VISIBLE_DEVICES") != "")
