@@ -11,6 +11,9 @@ no code with the CUDA path. Library primitives (``numpy.tensordot``, ``@``,
 ``scipy.special.erf``) serve as single steps; nothing is blocked, fused or
 reordered beyond the definitions.
 
+``sampler`` holds the noise schedules, the DDPM / DDIM reverse updates and
+classifier-free guidance that sit on either side of the denoiser step.
+
 Parity pins: see ``tests/test_oracle_*.py``. Every function here is pinned by
 at least one check that does not retype its own formula (brute-force loops,
 closed forms, invariants, page-printed shapes and parameter totals). The
@@ -22,6 +25,8 @@ from .ops import (bf16_round, group_norm, silu, conv2d, upsample_nearest2x, line
 from .model import (UNetConfig, SD21_BASE, SDXL_INPAINT, enumerate_unet_params,
                     enumerate_resblock_params, enumerate_transformer_params,
                     enumerate_time_mlp_params, time_mlp, resblock, transformer,
-                    downsample, upsample, conv_in, unet_step, unet_shapes)
+                    downsample, upsample, conv_in, unet_step, unet_stages, unet_shapes,
+                    add_embedding)
+from . import sampler
 
 __all__ = [n for n in dir() if not n.startswith("_")]

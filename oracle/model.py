@@ -58,11 +58,21 @@ class UNetConfig:
     temb_dim: int = 1280
     groups: int = 32
     eps: float = 1e-5
+    # SDXL added conditioning: a pooled text vector of add_text_dim values and
+    # add_time_ids scalars (original size, crop offset, target size), each
+    # Fourier-encoded to add_time_dim values like the timestep; 0 = none.
+    add_text_dim: int = 0
+    add_time_ids: int = 0
+    add_time_dim: int = 256
+
+    @property
+    def add_embed_dim(self) -> int:
+        return self.add_text_dim + self.add_time_ids * self.add_time_dim if self.add_text_dim else 0
 
 
 SD21_BASE = UNetConfig()
 SDXL_INPAINT = UNetConfig(in_channels=9, block_channels=(320, 640, 1280), attn_depth=(0, 2, 10),
-                          mid_depth=10, ctx_dim=2048)
+                          mid_depth=10, ctx_dim=2048, add_text_dim=1280, add_time_ids=6)
 
 
 # --------------------------------------------------------------------------- parameter tables
@@ -159,6 +169,8 @@ def enumerate_unet_params(cfg: UNetConfig = SD21_BASE):
     ch = cfg.block_channels
     L = len(ch)
     p = enumerate_time_mlp_params("time", cfg.time_proj_dim, cfg.temb_dim)
+    if cfg.add_embed_dim:
+        p += enumerate_time_mlp_params("add", cfg.add_embed_dim, cfg.temb_dim)
     p += enumerate_conv_params("conv_in", cfg.in_channels, ch[0])
     c_prev = ch[0]
     for lvl in range(L):
@@ -205,6 +217,22 @@ def time_mlp(params, t: float, prefix="time", proj_dim=320):
     Linear; tutorial page, time-embedding paragraphs)."""
     phi = timestep_embedding(t, proj_dim)[None, :]
     h = linear(phi, _w(params, f"{prefix}.lin1.weight"), _w(params, f"{prefix}.lin1.bias"))
+    h = linear(silu(h), _w(params, f"{prefix}.lin2.weight"), _w(params, f"{prefix}.lin2.bias"))
+    return h[0]
+
+
+def add_embedding(params, text, time_ids, cfg: UNetConfig, prefix="add"):
+    """SDXL added conditioning (tutorial page, SDXL conditioning paragraphs:
+    the image-size, crop and target-size conditions are Fourier-encoded like the
+    timestep and concatenated after the pooled text embedding, 2816 values for
+    SDXL): a = [text | phi(v_0) | ... | phi(v_5)], then the same
+    Linear -> SiLU -> Linear shape as the time MLP; the result is added to temb."""
+    parts = [np.asarray(text, dtype=np.float64).reshape(-1)]
+    for v in time_ids:
+        parts.append(timestep_embedding(float(v), cfg.add_time_dim))
+    a = np.concatenate(parts)[None, :]
+    assert a.shape[1] == cfg.add_embed_dim
+    h = linear(a, _w(params, f"{prefix}.lin1.weight"), _w(params, f"{prefix}.lin1.bias"))
     h = linear(silu(h), _w(params, f"{prefix}.lin2.weight"), _w(params, f"{prefix}.lin2.bias"))
     return h[0]
 
@@ -289,8 +317,12 @@ def conv_in(x, params, prefix="conv_in"):
     return conv2d(np.asarray(x, dtype=np.float64), _w(params, f"{prefix}.weight"), _w(params, f"{prefix}.bias"), 1, 1)
 
 
-def unet_step(latent, t, ctx, params, cfg: UNetConfig = SD21_BASE, record_shapes=None):
-    """One denoiser timestep: eps = UNet(latent [in_ch, H, W], t, ctx [77, D]).
+def unet_stages(latent, t, ctx, params, cfg: UNetConfig = SD21_BASE, add_text=None, add_time_ids=None,
+                record=None):
+    """The denoiser step as a sequence of modules: yields (name, output) after
+    the time embedding, conv_in, every resblock, transformer, resampling conv and
+    the output head, in forward order, and each up-path resblock's concatenated
+    input as "up.<u>.res.<i>.in"; the last item is ("out", eps).
 
     h = conv_in(latent), pushed; per level: layers_per_block resblocks (each
     followed by a transformer where the level has attention), each output
@@ -298,52 +330,70 @@ def unet_step(latent, t, ctx, params, cfg: UNetConfig = SD21_BASE, record_shapes
     resblock -> transformer -> resblock; per up level: layers_per_block + 1 times
     pop a skip, concatenate [h, skip] on channels, resblock (+ transformer), then
     a nearest-2x upsample conv (except the last up level); output
-    conv_out(SiLU(GN(h)))."""
+    conv_out(SiLU(GN(h))). With SDXL added conditioning the add embedding is
+    added to temb before any resblock uses it. ``record`` (a dict) receives
+    each block's sublayer outputs under the module's name."""
     ch = cfg.block_channels
     L = len(ch)
     G, eps = cfg.groups, cfg.eps
     temb = time_mlp(params, t, "time", cfg.time_proj_dim)
+    if cfg.add_embed_dim:
+        temb = temb + add_embedding(params, add_text, add_time_ids, cfg)
+    yield "temb", temb
     h = conv_in(latent, params, "conv_in")
+    yield "conv_in", h
     skips = [h]
-    rec = record_shapes
-    if rec is not None:
-        rec.append(("conv_in", h.shape))
     for lvl in range(L):
         for i in range(cfg.layers_per_block):
-            h = resblock(h, temb, params, f"down.{lvl}.res.{i}", G, eps)
+            h = resblock(h, temb, params, f"down.{lvl}.res.{i}", G, eps, record)
+            yield f"down.{lvl}.res.{i}", h
             if cfg.attn_depth[lvl] > 0:
-                h = transformer(h, ctx, params, f"down.{lvl}.attn.{i}", cfg.attn_depth[lvl], cfg.head_dim, G, eps, eps)
+                h = transformer(h, ctx, params, f"down.{lvl}.attn.{i}", cfg.attn_depth[lvl], cfg.head_dim, G, eps,
+                                eps, record)
+                yield f"down.{lvl}.attn.{i}", h
             skips.append(h)
-            if rec is not None:
-                rec.append((f"down.{lvl}.{i}", h.shape))
         if lvl < L - 1:
             h = downsample(h, params, f"down.{lvl}.down")
+            yield f"down.{lvl}.down", h
             skips.append(h)
-            if rec is not None:
-                rec.append((f"down.{lvl}.down", h.shape))
-    h = resblock(h, temb, params, "mid.res.0", G, eps)
-    h = transformer(h, ctx, params, "mid.attn.0", cfg.mid_depth, cfg.head_dim, G, eps, eps)
-    h = resblock(h, temb, params, "mid.res.1", G, eps)
-    if rec is not None:
-        rec.append(("mid", h.shape))
+    h = resblock(h, temb, params, "mid.res.0", G, eps, record)
+    yield "mid.res.0", h
+    h = transformer(h, ctx, params, "mid.attn.0", cfg.mid_depth, cfg.head_dim, G, eps, eps, record)
+    yield "mid.attn.0", h
+    h = resblock(h, temb, params, "mid.res.1", G, eps, record)
+    yield "mid.res.1", h
     for up in range(L):
         lvl = L - 1 - up
         for i in range(cfg.layers_per_block + 1):
             s = skips.pop()
-            if rec is not None:
-                rec.append((f"up.{up}.{i}.in", (h.shape[0] + s.shape[0],) + h.shape[1:]))
-            h = resblock(np.concatenate([h, s], axis=0), temb, params, f"up.{up}.res.{i}", G, eps)
+            h = np.concatenate([h, s], axis=0)
+            yield f"up.{up}.res.{i}.in", h
+            h = resblock(h, temb, params, f"up.{up}.res.{i}", G, eps, record)
+            yield f"up.{up}.res.{i}", h
             if cfg.attn_depth[lvl] > 0:
-                h = transformer(h, ctx, params, f"up.{up}.attn.{i}", cfg.attn_depth[lvl], cfg.head_dim, G, eps, eps)
+                h = transformer(h, ctx, params, f"up.{up}.attn.{i}", cfg.attn_depth[lvl], cfg.head_dim, G, eps, eps,
+                                record)
+                yield f"up.{up}.attn.{i}", h
         if up < L - 1:
             h = upsample(h, params, f"up.{up}.up")
-        if rec is not None:
-            rec.append((f"up.{up}", h.shape))
+            yield f"up.{up}.up", h
     assert not skips
     h = silu(group_norm(h, _w(params, "out.norm.gamma"), _w(params, "out.norm.beta"), G, eps))
     out = conv2d(h, _w(params, "conv_out.weight"), _w(params, "conv_out.bias"), 1, 1)
-    if rec is not None:
-        rec.append(("out", out.shape))
+    yield "out", out
+
+
+def unet_step(latent, t, ctx, params, cfg: UNetConfig = SD21_BASE, record_shapes=None, add_text=None,
+              add_time_ids=None, record=None):
+    """One denoiser timestep: eps = UNet(latent [in_ch, H, W], t, ctx [77, D])
+    (and the SDXL added conditioning when the config has it), the modules of
+    ``unet_stages`` run in order. ``record_shapes`` (a list) receives the
+    shape of every module output."""
+    out = None
+    for name, h in unet_stages(latent, t, ctx, params, cfg, add_text, add_time_ids, record):
+        if record_shapes is not None and name != "temb":
+            record_shapes.append((name, h.shape))
+        out = h
     return out
 
 

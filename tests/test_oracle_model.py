@@ -68,7 +68,13 @@ def test_unet_shape_walk_small_model():
     assert out.shape == (4, 16, 16)
     assert np.all(np.isfinite(out))
     skips, up_cin = model.unet_shapes(cfg, 16, 16)
-    pushed = [s for name, s in rec if name == "conv_in" or name.startswith("down.")]
+    shapes = dict(rec)
+    pushed = [shapes["conv_in"]]
+    for lvl in range(4):
+        for i in range(cfg.layers_per_block):
+            pushed.append(shapes.get(f"down.{lvl}.attn.{i}", shapes[f"down.{lvl}.res.{i}"]))
+        if lvl < 3:
+            pushed.append(shapes[f"down.{lvl}.down"])
     assert [tuple(s) for s in pushed] == [tuple(s) for s in skips]
     ins = [s[0] for name, s in rec if name.endswith(".in")]
     assert ins == up_cin
@@ -96,10 +102,15 @@ def test_sd21_param_total_matches_page():
 
 
 def test_sdxl_param_total_matches_page():
+    """U-Net with its 2816-d added-conditioning MLP (this enumerator) + both text
+    encoders + VAE round to the 3.469B of the SDXL-Inpainting page section 5."""
     g = load("sdxl_inpaint_topology.json")
-    unet = count(model.enumerate_unet_params(model.SDXL_INPAINT))
-    add_embedding = (2816 * 1280 + 1280) + (1280 * 1280 + 1280)  # not built: outside the scored configs
-    total = unet + add_embedding + g["clip_l_params_million"] * 1e6 + g["openclip_bigg_params_million"] * 1e6 \
+    table = model.enumerate_unet_params(model.SDXL_INPAINT)
+    unet = count(table)
+    add = [(n, s) for n, s, _, _ in table if n.startswith("add.")]
+    assert add[0][1] == (1280, 2816)  # pooled text 1280 + 6 Fourier-encoded size/crop values x 256
+    assert model.SDXL_INPAINT.add_embed_dim == 2816
+    total = unet + g["clip_l_params_million"] * 1e6 + g["openclip_bigg_params_million"] * 1e6 \
         + g["vae_fp16_file_mb"] * 1e6 / 2
     assert abs(total / 1e9 - g["params_total_billion"]) < 0.0006
 

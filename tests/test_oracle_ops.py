@@ -325,3 +325,28 @@ def test_bf16_round_known_values():
     assert r[0] == 1.0 and r[1] == 1.0
     assert r[2] == 1.0 + 2 ** -6  # tie between 1+2^-7 and 1+2^-6, rounds to even mantissa
     assert r[3] == 1.0 + 2 ** -7 and r[4] == -2.5
+
+
+# ----------------------------------------------------------------------------- SiLU
+
+@pytest.mark.parametrize("x,expected", [
+    (0.0, 0.0),
+    (1.0, 0.7310585786300049),    # 1 * logistic(1), tabulated
+    (-1.0, -0.2689414213699951),  # -1 * logistic(-1)
+    (2.0, 1.7615941559557649),    # 2 * logistic(2)
+    (-2.0, -0.2384058440442351),
+])
+def test_silu_tabulated(x, expected):
+    assert abs(float(ops.silu(np.array([x]))[0]) - expected) < 1e-15
+
+
+def test_silu_limits_and_even_part():
+    """SiLU(x) -> x for large x and -> 0 for very negative x; its even part
+    SiLU(x) + SiLU(-x) equals x * tanh(x / 2) (a sign slip, a dropped x or a
+    plain sigmoid breaks one of these)."""
+    big = np.array([30.0, 40.0])
+    np.testing.assert_allclose(ops.silu(big), big, rtol=1e-12)
+    assert np.all(np.abs(ops.silu(-big)) < 1e-11)
+    x = np.linspace(-6.0, 6.0, 49)
+    np.testing.assert_allclose(ops.silu(x) + ops.silu(-x), x * np.tanh(x / 2.0), atol=1e-14)
+    np.testing.assert_allclose(ops.silu(x) - ops.silu(-x), x, atol=1e-14)
