@@ -133,7 +133,13 @@ typedef struct {
   float ln_eps;      /* 1e-5 */
 } sd_transformer_cfg;
 
-/* Whole denoiser [SD21 section 3; SDXLI section 3]. */
+/* Whole denoiser [SD21 section 3; SDXLI section 3]. The three add_* fields
+ * describe SDXL's added conditioning [TUT, SDXL conditioning paragraphs]: a
+ * pooled text vector of add_text_dim values and add_time_ids scalars (original
+ * size, crop offset, target size), each Fourier-encoded like the timestep to
+ * add_time_dim values and concatenated after the text (1280 + 6 x 256 = 2816 for
+ * SDXL); that vector goes through Linear -> SiLU -> Linear (the time MLP's shape)
+ * and is added to the time embedding. add_text_dim = 0 disables it (SD2.1). */
 typedef struct {
   int32_t in_channels;        /* 4, or 9 for inpainting */
   int32_t out_channels;       /* 4 */
@@ -151,6 +157,9 @@ typedef struct {
   int32_t temb_dim;           /* 1280 */
   int32_t groups;             /* 32 */
   float eps;                  /* 1e-5, for every GroupNorm and LayerNorm */
+  int32_t add_text_dim;       /* 0 = no added conditioning; 1280 for SDXL */
+  int32_t add_time_ids;       /* 0..8 scalars (6 for SDXL) */
+  int32_t add_time_dim;       /* Fourier width per scalar (256 for SDXL), even */
 } sd_unet_cfg;
 
 /* ---------------------------------------------------------------- weights (host only) */
@@ -176,9 +185,18 @@ sd_status sd_unet_weight_layout(const sd_unet_cfg* cfg, sd_tensor_desc* out, int
 enum { SD_CONV_IN = 0, SD_CONV_DOWNSAMPLE = 1, SD_CONV_UPSAMPLE = 2, SD_CONV_OUTPUT = 3 };
 
 /* Convert a canonical BF16 buffer (host, uint16 bit patterns) into the packed
- * layout (host buffer of packed_bytes). Conv weights become [O][ky][kx][C]; the
- * GEGLU FF1 rows are interleaved (value j, gate j); everything else is copied.
- * Each tensor starts on a 256-byte boundary. */
+ * layout (host buffer of packed_bytes); host code only, no stream. Each tensor
+ * starts on a 256-byte boundary, in table order:
+ *   - 3x3 conv weights become [O][ky][kx][C]; conv_in weights become [O][Kp] in
+ *     im2col order k = (ky*3 + kx)*C + c, zero-padded to a multiple of 64;
+ *   - the three linear layers fed by a LayerNorm in each BasicTransformer block
+ *     (attn1 q/k/v, attn2 q, ff.w1) are stored multiplied by that LayerNorm's
+ *     gamma along K and rounded to BF16 (W' = W * gamma); ff.w1 rows and bias are
+ *     also interleaved (value j, gate j);
+ *   - after each block's tensors come two derived FP32 vectors per such layer:
+ *     c1 = row sums of W' and c2 = W * beta + bias, which the GEMM epilogue uses
+ *     to apply the LayerNorm from per-row statistics (no LayerNorm kernel runs);
+ *   - every other tensor is copied unchanged. */
 sd_status sd_time_pack_weights(const sd_time_cfg* cfg, const uint16_t* canonical, void* packed);
 sd_status sd_conv_pack_weights(const sd_conv_cfg* cfg, int32_t conv_kind, const uint16_t* canonical,
                                void* packed);
@@ -212,12 +230,14 @@ sd_status sd_time_embed(const sd_time_cfg* cfg, const void* packed_w, float time
  * (2 x 4096 FP32 = 32 KiB, resident on every GPU that loads the library until
  * the process exits). proj_dim and temb_dim above 4096 are rejected with
  * SD_ERR_UNSUPPORTED before anything is launched. No device or host memory is
- * allocated. The first call on a device looks up that array's device address
- * (with the device current), so make the first call on each device before any
- * stream capture. All calls share the one array: calls whose work overlaps on
- * the GPU (different streams, or different host threads, without ordering)
- * race on it; serialise them. Each call rewrites both vectors before reading
- * them, so no state carries over between calls. */
+ * allocated. Every call looks up that array's device address on the current
+ * device (a host-side query, so the address stays right after a device reset);
+ * the first lookup on a device may load the library's device code, so make the
+ * first call on each device before any stream capture. All calls share the one
+ * array: calls whose work overlaps on the GPU (different streams, or different
+ * host threads, without ordering) race on it; serialise them. Each call
+ * rewrites both vectors before reading them, so no state carries over between
+ * calls. */
 sd_status sd_time_embed_noalloc(const sd_time_cfg* cfg, const void* packed_w, float timestep, float* temb_out,
                                 sd_stream_t stream);
 
@@ -247,10 +267,21 @@ sd_status sd_transformer_fwd(const sd_transformer_cfg* cfg, const void* packed_w
 /* One denoiser timestep. latent: [H, W, in_channels] BF16 (for in_channels = 9
  * the caller passes the assembled 9-channel input), context [ctx_len, ctx_dim],
  * eps_out [H, W, out_channels]. The skip stack and every intermediate live in
- * the workspace. */
+ * the workspace. A config with added conditioning (add_text_dim > 0) needs
+ * sd_unet_step_cond; here it returns SD_ERR_NULL_ARG. */
 sd_status sd_unet_step(const sd_unet_cfg* cfg, const void* packed_w, const void* latent, float timestep,
                        const void* context, void* eps_out, void* workspace, size_t ws_bytes,
                        sd_stream_t stream);
+
+/* sd_unet_step with SDXL's added conditioning [TUT, SDXL conditioning
+ * paragraphs; SDXLI section 1]: add_text = device BF16 [add_text_dim] pooled
+ * text vector; add_time_ids = HOST array of add_time_ids floats (SDXL: original
+ * height, width, crop top, left, target height, width), read during this call
+ * (a captured graph keeps the values it was captured with). Both may be NULL
+ * when cfg->add_text_dim is 0. */
+sd_status sd_unet_step_cond(const sd_unet_cfg* cfg, const void* packed_w, const void* latent, float timestep,
+                            const void* context, const void* add_text, const float* add_time_ids, void* eps_out,
+                            void* workspace, size_t ws_bytes, sd_stream_t stream);
 
 /* Synchronises `stream`, then reads the device error word of `workspace`:
  * SD_OK, or SD_ERR_DEVICE_TIMEOUT when a bounded wait gave up; the word is
@@ -299,6 +330,46 @@ sd_status sd_profile_read(sd_launch_record* out, int32_t capacity, int32_t* n);
  * against calls in flight on other host threads. The pages have no
  * counterpart: this only selects among equivalent schedules. */
 sd_status sd_gemm_override(int32_t bn, int32_t splits);
+
+/* ---------------------------------------------------------------- sublayer record (testing)
+ * Per calling thread: between sd_record_begin() and sd_record_end(), every
+ * ResnetBlock2D and Transformer2DModel this library runs also writes the
+ * outputs of its sublayers BEFORE their residual add into `dev_buf` (caller-
+ * owned device memory of `bytes` bytes), as BF16 token matrices:
+ *   "h1"    conv1(SiLU(GN1(x))) + b1 + time projection of a resblock [HW, C_out];
+ *   "attn1" the self-attention output after its out-projection and bias [HW, C];
+ *   "attn2" the same for the cross-attention;
+ *   "ff"    the GEGLU feed-forward output after its second linear and bias.
+ * These are the intermediate values of [SD21 section 4]'s block panels, for
+ * comparing each sublayer with a reference. The extra outputs are computed by
+ * extra launches enqueued on the call's stream (the normal outputs are
+ * unchanged). `module` counts resblocks ("h1") or transformers (the others) in
+ * the order they ran since sd_record_begin; `block` is the BasicTransformer block.
+ * An entry that no longer fits is dropped and sd_record_end returns
+ * SD_ERR_CAPACITY. */
+typedef struct {
+  char name[8];    /* "h1", "attn1", "attn2", "ff" */
+  int32_t module;
+  int32_t block;
+  int64_t offset;  /* byte offset in dev_buf */
+  int64_t rows;    /* tokens (H*W) */
+  int64_t cols;    /* channels */
+} sd_record_entry;
+
+sd_status sd_record_begin(void* dev_buf, size_t bytes);
+sd_status sd_record_end(int32_t* n_entries);
+sd_status sd_record_read(sd_record_entry* out, int32_t capacity, int32_t* n);
+
+/* Test hook for the device-side timeout path (the pages have no counterpart).
+ * The next n_launches tensor-core GEMM kernels enqueued by this process first
+ * make one thread of every CTA wait on a barrier that nothing completes, for
+ * at most spin_limit polls (1 .. 2^24); the wait gives up, raises the device
+ * error flag in the workspace header and makes every role of the CTA skip its
+ * work, so the kernel loads nothing, computes nothing, writes no output (the
+ * output buffer keeps stale values) and releases its tensor memory before it
+ * returns. sd_query_device_status then reports SD_ERR_DEVICE_TIMEOUT.
+ * n_launches = 0 cancels. Process-wide. */
+sd_status sd_debug_inject_timeout(int32_t n_launches, int32_t spin_limit);
 
 /* Kernel launches issued by this library in this process so far. */
 int64_t sd_launch_count(void);

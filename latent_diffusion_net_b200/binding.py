@@ -60,7 +60,13 @@ class sd_unet_cfg(ctypes.Structure):
                 ("n_levels", c_int32), ("block_channels", c_int32 * 4), ("attn_depth", c_int32 * 4),
                 ("layers_per_block", c_int32), ("mid_depth", c_int32), ("head_dim", c_int32),
                 ("ctx_len", c_int32), ("ctx_dim", c_int32), ("time_proj_dim", c_int32), ("temb_dim", c_int32),
-                ("groups", c_int32), ("eps", c_float)]
+                ("groups", c_int32), ("eps", c_float), ("add_text_dim", c_int32), ("add_time_ids", c_int32),
+                ("add_time_dim", c_int32)]
+
+
+class sd_record_entry(ctypes.Structure):
+    _fields_ = [("name", c_char * 8), ("module", c_int32), ("block", c_int32), ("offset", c_int64),
+                ("rows", c_int64), ("cols", c_int64)]
 
 
 class sd_launch_record(ctypes.Structure):
@@ -101,6 +107,12 @@ _SIGS = {
     "sd_resblock_fwd": (c_int32, [POINTER(sd_resblock_cfg), _P, _P, _P, _P, _P, _P, c_size_t, _P]),
     "sd_transformer_fwd": (c_int32, [POINTER(sd_transformer_cfg), _P, _P, _P, _P, _P, c_size_t, _P]),
     "sd_unet_step": (c_int32, [POINTER(sd_unet_cfg), _P, _P, c_float, _P, _P, _P, c_size_t, _P]),
+    "sd_unet_step_cond": (c_int32, [POINTER(sd_unet_cfg), _P, _P, c_float, _P, _P, POINTER(c_float), _P, _P,
+                                    c_size_t, _P]),
+    "sd_record_begin": (c_int32, [_P, c_size_t]),
+    "sd_record_end": (c_int32, [POINTER(c_int32)]),
+    "sd_record_read": (c_int32, [POINTER(sd_record_entry), c_int32, POINTER(c_int32)]),
+    "sd_debug_inject_timeout": (c_int32, [c_int32, c_int32]),
     "sd_query_device_status": (c_int32, [_P, _P]),
     "sd_profile_begin": (c_int32, []),
     "sd_profile_end": (c_int32, [POINTER(c_int32)]),
@@ -290,6 +302,45 @@ def sd_unet_step(cfg, packed_w, latent, timestep, context, eps_out, workspace, w
     return _check(s, "sd_unet_step") if check else s
 
 
+def sd_unet_step_cond(cfg, packed_w, latent, timestep, context, add_text, add_time_ids, eps_out, workspace,
+                      ws_bytes, stream=None, check=True):
+    """add_time_ids: a sequence of host floats (or None)."""
+    ids = None
+    if add_time_ids is not None:
+        vals = [float(v) for v in add_time_ids]
+        ids = (c_float * max(len(vals), 1))(*vals)
+    s = lib().sd_unet_step_cond(ctypes.byref(cfg), _ptr(packed_w), _ptr(latent), float(timestep), _ptr(context),
+                                _ptr(add_text), ids, _ptr(eps_out), _ptr(workspace), int(ws_bytes), _stream(stream))
+    return _check(s, "sd_unet_step_cond") if check else s
+
+
+def sd_record_begin(dev_buf, nbytes):
+    return _check(lib().sd_record_begin(_ptr(dev_buf), int(nbytes)), "sd_record_begin")
+
+
+def sd_record_end(check=True):
+    """Returns (status, number of entries)."""
+    n = c_int32(0)
+    s = lib().sd_record_end(ctypes.byref(n))
+    if check:
+        _check(s, "sd_record_end")
+    return s, n.value
+
+
+def sd_record_read():
+    """Entries of the last recording: list of dicts (name, module, block, offset, rows, cols)."""
+    n = c_int32(0)
+    _check(lib().sd_record_read(None, 0, ctypes.byref(n)), "sd_record_read")
+    arr = (sd_record_entry * max(n.value, 1))()
+    _check(lib().sd_record_read(arr, n.value, ctypes.byref(n)), "sd_record_read")
+    return [{"name": e.name.decode(), "module": e.module, "block": e.block, "offset": e.offset, "rows": e.rows,
+             "cols": e.cols} for e in arr[:n.value]]
+
+
+def sd_debug_inject_timeout(n_launches, spin_limit=1024):
+    return _check(lib().sd_debug_inject_timeout(int(n_launches), int(spin_limit)), "sd_debug_inject_timeout")
+
+
 def sd_query_device_status(workspace, stream=None):
     return lib().sd_query_device_status(_ptr(workspace), _stream(stream))
 
@@ -343,9 +394,20 @@ def transformer_cfg(height, width, channels, depth=1, ctx_len=77, ctx_dim=1024, 
 
 def unet_cfg(in_channels=4, out_channels=4, height=96, width=96, block_channels=(320, 640, 1280, 1280),
              attn_depth=(1, 1, 1, 0), layers_per_block=2, mid_depth=1, ctx_len=77, ctx_dim=1024,
-             time_proj_dim=320, temb_dim=1280, groups=32, eps=1e-5):
+             time_proj_dim=320, temb_dim=1280, groups=32, eps=1e-5, add_text_dim=0, add_time_ids=0,
+             add_time_dim=256):
     bc = list(block_channels) + [0] * (4 - len(block_channels))
     ad = list(attn_depth) + [0] * (4 - len(attn_depth))
     return sd_unet_cfg(in_channels, out_channels, height, width, len(block_channels), (c_int32 * 4)(*bc),
                        (c_int32 * 4)(*ad), layers_per_block, mid_depth, 64, ctx_len, ctx_dim, time_proj_dim,
-                       temb_dim, groups, eps)
+                       temb_dim, groups, eps, add_text_dim, add_time_ids, add_time_dim)
+
+
+def unet_cfg_from(ocfg, height, width):
+    """C config of an oracle UNetConfig (same field names)."""
+    return unet_cfg(in_channels=ocfg.in_channels, out_channels=ocfg.out_channels, height=height, width=width,
+                    block_channels=ocfg.block_channels, attn_depth=ocfg.attn_depth,
+                    layers_per_block=ocfg.layers_per_block, mid_depth=ocfg.mid_depth, ctx_len=ocfg.ctx_len,
+                    ctx_dim=ocfg.ctx_dim, time_proj_dim=ocfg.time_proj_dim, temb_dim=ocfg.temb_dim,
+                    groups=ocfg.groups, eps=ocfg.eps, add_text_dim=ocfg.add_text_dim,
+                    add_time_ids=ocfg.add_time_ids, add_time_dim=ocfg.add_time_dim)

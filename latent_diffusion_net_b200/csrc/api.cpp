@@ -146,6 +146,42 @@ sd_status run_gn(const Ctx& c, const bf16* x0, int C0, const bf16* x1, int C1, i
   return SD_OK;
 }
 
+// Sublayer record (sd_record_*): per calling thread.
+struct Recorder {
+  bool on = false;
+  uint8_t* buf = nullptr;
+  size_t bytes = 0, used = 0;
+  bool overflow = false;
+  int res_count = 0, tx_count = 0;
+  std::vector<sd_record_entry> entries;
+};
+thread_local Recorder t_rec;
+
+// Device slot for one recorded [rows][cols] BF16 matrix, or null when it does not fit.
+bf16* rec_slot(const char* name, int module, int block, int64_t rows, int64_t cols) {
+  Recorder& r = t_rec;
+  const size_t off = (r.used + 255) & ~size_t(255);
+  const size_t need = (size_t)rows * cols * 2;
+  if (off + need > r.bytes) {
+    r.overflow = true;
+    return nullptr;
+  }
+  sd_record_entry e;
+  memset(&e, 0, sizeof(e));
+  strncpy(e.name, name, sizeof(e.name) - 1);
+  e.module = module;
+  e.block = block;
+  e.offset = (int64_t)off;
+  e.rows = rows;
+  e.cols = cols;
+  r.entries.push_back(e);
+  r.used = off + need;
+  return reinterpret_cast<bf16*>(r.buf + off);
+}
+
+// Timeout injection for tests (sd_debug_inject_timeout).
+std::atomic<int> g_inject_n{0}, g_inject_spins{0};
+
 // Launch a GEMM problem under a profiling scope with its algorithmic work:
 // FLOPs 2*M*N*K (K = reduction length; alg_k overrides a zero-padded K), bytes
 // = every A source and B matrix read once, the output (and residual) once.
@@ -155,6 +191,8 @@ int launch_gemm(const Ctx& c, const GemmProblem& p0, double alg_k = 0) {
   GemmProblem p = p0;
   p.force_bn = g_force_bn.load(std::memory_order_relaxed);
   p.force_splits = g_force_splits.load(std::memory_order_relaxed);
+  if (g_inject_n.load(std::memory_order_relaxed) > 0 && g_inject_n.fetch_sub(1) > 0)
+    p.hold_spins = g_inject_spins.load(std::memory_order_relaxed);
   double K = 0;
   for (int i = 0; i < p.nseg; ++i) K += 64.0 * p.seg[i].nkb;
   if (alg_k > 0) K = alg_k;
@@ -210,7 +248,7 @@ struct LnFold {
 
 sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, int N, const bf16* bias,
                      const bf16* residual, int ld_res, bf16* out, int ld_out, int mode = sdk::GEMM_PLAIN,
-                     double alg_k = 0, int f16_begin = 0, const LnFold* ln = nullptr) {
+                     double alg_k = 0, const LnFold* ln = nullptr) {
   GemmProblem p = base_problem(c);
   p.Ho = 1;
   p.Wo = M;
@@ -227,7 +265,6 @@ sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, i
   p.epi.out = out;
   p.epi.ld_out = ld_out;
   p.epi.mode = mode;
-  p.epi.f16_begin = f16_begin;
   if (ln) {
     p.epi.rowstat_out = ln->out;
     p.epi.rowstat_clear = ln->clear;
@@ -279,6 +316,7 @@ sd_status run_resblock(const Ctx& c, const ResW& w, const void* pw, int H, int W
   const int HW = H * Wd;
   const int cin = cx + cs;
   const int cout = w.c_out;
+  const int rmod = t_rec.on ? t_rec.res_count++ : -1;
   sd_status r;
   // h1 = conv1(SiLU(GN1([x | skip]))) + b1 + tproj
   if ((r = run_gn(c, x, cx, skip, cs, HW, G, eps, W(pw, w.n1g), W(pw, w.n1b), 1, s.xn)) != SD_OK) return r;
@@ -297,6 +335,11 @@ sd_status run_resblock(const Ctx& c, const ResW& w, const void* pw, int H, int W
     p.epi.out = s.h1;
     p.epi.ld_out = cout;
     CK(launch_gemm(c, p));
+  }
+  if (rmod >= 0) {
+    bf16* d = rec_slot("h1", rmod, 0, HW, cout);
+    if (d && cudaMemcpyAsync(d, s.h1, (size_t)HW * cout * 2, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+      return SD_ERR_LAUNCH;
   }
   // y = conv2(SiLU(GN2(h1))) + b2 + shortcut
   if ((r = run_gn(c, s.h1, cout, nullptr, 0, HW, G, eps, W(pw, w.n2g), W(pw, w.n2b), 1, s.hn)) != SD_OK) return r;
@@ -366,6 +409,15 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
   const int C = w.C;
   const int heads = C / 64;
   if (!c.rs[0] || !c.rs_clean || c.rs_rows < HW) return SD_ERR_UNSUPPORTED;
+  const int tmod = t_rec.on ? t_rec.tx_count++ : -1;
+  int bi = 0;  // BasicTransformer block index
+  // recorded sublayer output before its residual add: the same linear layer without the residual
+  auto record = [&](const char* name, const bf16* A, int K, int64_t w_off, int64_t b_off) -> sd_status {
+    if (tmod < 0) return SD_OK;
+    bf16* d = rec_slot(name, tmod, bi, HW, C);
+    if (!d) return SD_OK;
+    return run_linear(c, A, HW, K, W(pw, w_off), C, W(pw, b_off), nullptr, 0, d, C);
+  };
   // The three LayerNorms of each block are folded into the GEMMs they feed
   // (Q/K/V, the cross-attention query, FF1): every GEMM that writes the
   // residual stream t also leaves t's row sums in one of two buffers, and
@@ -400,7 +452,7 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
     // the other buffer is not known to be zero yet: clear it too
     LnFold f = producer();
     f.clear = c.rs[clean];
-    if ((r = run_linear(c, s.nrm, HW, C, W(pw, w.piw), C, W(pw, w.pib), nullptr, 0, s.t, C, sdk::GEMM_PLAIN, 0, 0,
+    if ((r = run_linear(c, s.nrm, HW, C, W(pw, w.piw), C, W(pw, w.pib), nullptr, 0, s.t, C, sdk::GEMM_PLAIN, 0,
                         &f)) != SD_OK)
       return r;
   }
@@ -409,29 +461,31 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
     {
       const LnFold f = consumer(b.qkv_c1, b.qkv_c2);
       if ((r = run_linear(c, s.t, HW, C, W(pw, b.qkv), 3 * C, nullptr, nullptr, 0, s.big, 3 * C, sdk::GEMM_PLAIN, 0,
-                          0, &f)) != SD_OK)
+                          &f)) != SD_OK)
         return r;
     }
     CK(run_attn(c, s.big, 3 * C, 0, s.big, 3 * C, C, 2 * C, s.ao, C, HW, HW, heads));
+    if ((r = record("attn1", s.ao, C, b.o1w, b.o1b)) != SD_OK) return r;
     {
       const LnFold f = producer();
-      if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o1w), C, W(pw, b.o1b), s.t, C, s.t, C, sdk::GEMM_PLAIN, 0, 0,
+      if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o1w), C, W(pw, b.o1b), s.t, C, s.t, C, sdk::GEMM_PLAIN, 0,
                           &f)) != SD_OK)
         return r;
     }
     // cross-attention: t += Wo' Attn(LN2(t), ctx)
     {
       const LnFold f = consumer(b.q2_c1, b.q2_c2);
-      if ((r = run_linear(c, s.t, HW, C, W(pw, b.q2), C, nullptr, nullptr, 0, s.big, C, sdk::GEMM_PLAIN, 0, 0, &f)) !=
+      if ((r = run_linear(c, s.t, HW, C, W(pw, b.q2), C, nullptr, nullptr, 0, s.big, C, sdk::GEMM_PLAIN, 0, &f)) !=
           SD_OK)
         return r;
     }
     if ((r = run_linear(c, ctx, ctx_len, w.ctx_dim, W(pw, b.kv2), 2 * C, nullptr, nullptr, 0, s.kv, 2 * C)) != SD_OK)
       return r;
     CK(run_attn(c, s.big, C, 0, s.kv, 2 * C, 0, C, s.ao, C, HW, ctx_len, heads));
+    if ((r = record("attn2", s.ao, C, b.o2w, b.o2b)) != SD_OK) return r;
     {
       const LnFold f = producer();
-      if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o2w), C, W(pw, b.o2b), s.t, C, s.t, C, sdk::GEMM_PLAIN, 0, 0,
+      if ((r = run_linear(c, s.ao, HW, C, W(pw, b.o2w), C, W(pw, b.o2b), s.t, C, s.t, C, sdk::GEMM_PLAIN, 0,
                           &f)) != SD_OK)
         return r;
     }
@@ -439,15 +493,17 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
     {
       const LnFold f = consumer(b.f1_c1, b.f1_c2);
       if ((r = run_linear(c, s.t, HW, C, W(pw, b.f1w), 8 * C, nullptr, nullptr, 0, s.big, 4 * C, sdk::GEMM_GEGLU, 0,
-                          0, &f)) != SD_OK)
-        return r;
-    }
-    {
-      const LnFold f = producer();
-      if ((r = run_linear(c, s.big, HW, 4 * C, W(pw, b.f2w), C, W(pw, b.f2b), s.t, C, s.t, C, sdk::GEMM_PLAIN, 0, 0,
                           &f)) != SD_OK)
         return r;
     }
+    if ((r = record("ff", s.big, 4 * C, b.f2w, b.f2b)) != SD_OK) return r;
+    {
+      const LnFold f = producer();
+      if ((r = run_linear(c, s.big, HW, 4 * C, W(pw, b.f2w), C, W(pw, b.f2b), s.t, C, s.t, C, sdk::GEMM_PLAIN, 0,
+                          &f)) != SD_OK)
+        return r;
+    }
+    ++bi;
   }
   *c.rs_clean = clean;
   // y = x + proj_out(t)
@@ -602,6 +658,12 @@ sd_status check_unet(const sd_unet_cfg* cfg) {
   if (cfg->time_proj_dim <= 0 || cfg->time_proj_dim % 16 || cfg->temb_dim <= 0 || cfg->temb_dim % 8)
     return SD_ERR_BAD_SHAPE;
   if (cfg->layers_per_block + 1 > 8) return SD_ERR_UNSUPPORTED;
+  if (cfg->add_text_dim < 0 || cfg->add_time_ids < 0 || cfg->add_time_ids > sdk::kMaxAddIds) return SD_ERR_UNSUPPORTED;
+  if (cfg->add_text_dim > 0) {
+    if (cfg->add_time_ids > 0 && (cfg->add_time_dim <= 0 || cfg->add_time_dim % 2)) return SD_ERR_BAD_SHAPE;
+    const int d = cfg->add_text_dim + cfg->add_time_ids * cfg->add_time_dim;
+    if (d % 8 || d > 16384) return SD_ERR_UNSUPPORTED;  // 16-byte weight rows in the GEMV; x staged in shared memory
+  }
   for (int l = 0; l < L; ++l) {
     if (!ch_ok(cfg->block_channels[l]) || cfg->block_channels[l] > 2048) return SD_ERR_UNSUPPORTED;
     if (!groups_ok(cfg->block_channels[l], cfg->groups) || cfg->attn_depth[l] < 0) return SD_ERR_UNSUPPORTED;
@@ -664,6 +726,7 @@ size_t plan_time(Arena& ar, const sd_time_cfg* cfg, cudaStream_t st, int sms, Ti
 struct UNetPlan {
   Ctx c;
   float *phi, *hid, *temb, *tproj;
+  float *add_x, *add_h;  // SDXL added conditioning: MLP input and hidden layer
   std::vector<bf16*> skip;      // 1 + L*lpb + (L-1) slots, push order
   std::vector<int> skip_c, skip_hw;
   bf16 *pp[2];                  // up-path ping-pong
@@ -680,6 +743,11 @@ size_t plan_unet(Arena& ar, const sd_unet_cfg* cfg, cudaStream_t st, int sms, UN
   p->phi = ar.f32(cfg->time_proj_dim);
   p->hid = ar.f32(cfg->temb_dim);
   p->temb = ar.f32(cfg->temb_dim);
+  p->add_x = p->add_h = nullptr;
+  if (cfg->add_text_dim > 0) {
+    p->add_x = ar.f32((size_t)cfg->add_text_dim + (size_t)cfg->add_time_ids * cfg->add_time_dim);
+    p->add_h = ar.f32(cfg->temb_dim);
+  }
   int64_t tsum = 0;
   for (int l = 0; l < L; ++l) tsum += (int64_t)ch[l] * (2 * cfg->layers_per_block + 1);
   tsum += 2 * ch[L - 1];
@@ -1082,10 +1150,19 @@ sd_status sd_transformer_fwd(const sd_transformer_cfg* cfg, const void* pw, cons
 
 sd_status sd_unet_step(const sd_unet_cfg* cfg, const void* pw, const void* latent, float timestep,
                        const void* context, void* eps_out, void* ws, size_t ws_bytes, sd_stream_t stream) {
+  return sd_unet_step_cond(cfg, pw, latent, timestep, context, nullptr, nullptr, eps_out, ws, ws_bytes, stream);
+}
+
+sd_status sd_unet_step_cond(const sd_unet_cfg* cfg, const void* pw, const void* latent, float timestep,
+                            const void* context, const void* add_text, const float* add_time_ids, void* eps_out,
+                            void* ws, size_t ws_bytes, sd_stream_t stream) {
   sd_status s = check_unet(cfg);
   if (s != SD_OK) return s;
   if (!pw || !latent || !context || !eps_out) return SD_ERR_NULL_ARG;
-  if (!aligned16(pw) || !aligned16(latent) || !aligned16(context) || !aligned16(eps_out)) return SD_ERR_MISALIGNED;
+  if (cfg->add_text_dim > 0 && (!add_text || (cfg->add_time_ids > 0 && !add_time_ids))) return SD_ERR_NULL_ARG;
+  if (!aligned16(pw) || !aligned16(latent) || !aligned16(context) || !aligned16(eps_out) ||
+      (add_text && cfg->add_text_dim > 0 && !aligned16(add_text)))
+    return SD_ERR_MISALIGNED;
   if ((s = check_ws(sd_unet_workspace_size(cfg), ws, ws_bytes)) != SD_OK) return s;
   DevInfo d;
   if ((s = device_info(&d)) != SD_OK) return s;
@@ -1110,6 +1187,32 @@ sd_status sd_unet_step(const sd_unet_cfg* cfg, const void* pw, const void* laten
   // time embedding and every resblock's projection of SiLU(temb), batched
   if ((s = run_time(c, u.time, pw, cfg->time_proj_dim, cfg->temb_dim, timestep, p.phi, p.hid, p.temb)) != SD_OK)
     return s;
+  if (u.has_add) {
+    // temb += Linear(SiLU(Linear([text | phi(id_0) | ...])))
+    sdk::AddIds ids;
+    memset(&ids, 0, sizeof(ids));
+    for (int i = 0; i < cfg->add_time_ids; ++i) ids.v[i] = add_time_ids[i];
+    const int dim = cfg->add_text_dim + cfg->add_time_ids * cfg->add_time_dim;
+    {
+      sdp::Scope sc("add_embed_input", sdp::F_OTHER, 0, 2.0 * cfg->add_text_dim + 4.0 * dim, c.st);
+      CK(sdk::launch_add_embed_input(static_cast<const bf16*>(add_text), cfg->add_text_dim, ids, cfg->add_time_ids,
+                                     cfg->add_time_dim, p.add_x, c.st));
+    }
+    sdk::GemvBatch b;
+    memset(&b, 0, sizeof(b));
+    b.njobs = 1;
+    b.K = dim;
+    b.silu_out = 1;
+    b.x = p.add_x;
+    b.job[0] = {W(pw, u.add.l1w), W(pw, u.add.l1b), p.add_h, cfg->temb_dim};
+    CK(run_gemv(c, b));
+    b.K = cfg->temb_dim;
+    b.silu_out = 0;
+    b.accum_out = 1;
+    b.x = p.add_h;
+    b.job[0] = {W(pw, u.add.l2w), W(pw, u.add.l2b), p.temb, cfg->temb_dim};
+    CK(run_gemv(c, b));
+  }
   std::vector<const ResW*> all_res;
   for (auto& lv : u.down)
     for (auto& r : lv.res) all_res.push_back(&r);
@@ -1213,6 +1316,43 @@ sd_status sd_unet_step(const sd_unet_cfg* cfg, const void* pw, const void* laten
   }
   return run_output(c, u.out, pw, H, Wd, hc, cfg->out_channels, G, eps, h, static_cast<bf16*>(eps_out),
                     reinterpret_cast<bf16*>(shared));
+}
+
+sd_status sd_record_begin(void* dev_buf, size_t bytes) {
+  if (!dev_buf && bytes) return SD_ERR_NULL_ARG;
+  if (!aligned16(dev_buf)) return SD_ERR_MISALIGNED;
+  Recorder& r = t_rec;
+  r.on = true;
+  r.buf = static_cast<uint8_t*>(dev_buf);
+  r.bytes = bytes;
+  r.used = 0;
+  r.overflow = false;
+  r.res_count = r.tx_count = 0;
+  r.entries.clear();
+  return SD_OK;
+}
+
+sd_status sd_record_end(int32_t* n_entries) {
+  Recorder& r = t_rec;
+  r.on = false;
+  if (n_entries) *n_entries = (int32_t)r.entries.size();
+  return r.overflow ? SD_ERR_CAPACITY : SD_OK;
+}
+
+sd_status sd_record_read(sd_record_entry* out, int32_t capacity, int32_t* n) {
+  const Recorder& r = t_rec;
+  if (n) *n = (int32_t)r.entries.size();
+  if (!out) return SD_OK;
+  if (capacity < (int32_t)r.entries.size()) return SD_ERR_CAPACITY;
+  for (size_t i = 0; i < r.entries.size(); ++i) out[i] = r.entries[i];
+  return SD_OK;
+}
+
+sd_status sd_debug_inject_timeout(int32_t n_launches, int32_t spin_limit) {
+  if (n_launches < 0 || (n_launches > 0 && (spin_limit < 1 || spin_limit > (1 << 24)))) return SD_ERR_UNSUPPORTED;
+  g_inject_spins.store(spin_limit, std::memory_order_relaxed);
+  g_inject_n.store(n_launches, std::memory_order_relaxed);
+  return SD_OK;
 }
 
 sd_status sd_query_device_status(void* ws, sd_stream_t stream) {

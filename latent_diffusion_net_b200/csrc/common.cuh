@@ -56,11 +56,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
 
 // ------------------------------------------------------------------ mbarrier
@@ -95,13 +90,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait: returns false (and raises the error flag) if the phase never
-// completes or if another thread of the CTA already gave up (*abort != 0).
+// completes within `limit` polls or if another thread of the CTA already gave
+// up (*abort != 0).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* err) {
+                                          int* err, uint32_t limit = kSpinLimit) {
   uint32_t n = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
-    if (++n > kSpinLimit) {
+    if (++n > limit) {
       *abort = 1;
       if (err) atomicOr(err, ERR_MBAR_TIMEOUT);
       return false;

@@ -54,6 +54,7 @@ struct GemmArgs {
   GemmEpi epi;
   float* partial;  // split-K: FP32 [splits][Ho*Wo][N]; null otherwise
   int* err;
+  int32_t hold_spins;  // tests only: see GemmProblem::hold_spins
 };
 
 __device__ __forceinline__ float gelu_erf(float g) { return 0.5f * g * (1.0f + erff(g * 0.70710678118654752f)); }
@@ -151,7 +152,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* acc_full = empty_bar + STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;       // [2], used in the even CTA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* hold_bar = acc_empty + 2;       // never completed (timeout test)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hold_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* epi_col = reinterpret_cast<float*>(smem + STAGES * stage_bytes + 256);  // [2][256] added terms
   float* epi_scl = epi_col + 512;                                                // [2][256] LayerNorm colscale
@@ -171,6 +173,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     mbar_init(&acc_full[1], 1);
     mbar_init(&acc_empty[0], 2);
     mbar_init(&acc_empty[1], 2);
+    mbar_init(hold_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -189,9 +192,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += (int64_t)gridDim.x * blockDim.x)
       z[i] = make_ulonglong2(0ull, 0ull);
   }
+  if (args.hold_spins > 0) {
+    // timeout test: nothing ever arrives on hold_bar, so this bounded wait gives
+    // up, raises the error flag and sets abort_flag; every role below then
+    // skips its work (no load is issued, so none is in flight at the teardown)
+    if (threadIdx.x == 0) mbar_wait(hold_bar, 0, abort_flag, args.err, (uint32_t)args.hold_spins);
+    __syncthreads();
+  }
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (lane == 0 && !*abort_flag) {
       for (int i = 0; i < kGemmMaxA; ++i) {
         tma_prefetch_desc(&maps.a[i]);
         tma_prefetch_desc(&maps.at[i]);
@@ -253,7 +263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+    if (lane == 0 && rank == 0 && !*abort_flag) {
       const uint32_t view_bytes = (uint32_t)args.BW * kBK * 2;  // one pixel row of the tall box
       int s = 0;
       uint32_t ph = 0;
@@ -317,7 +327,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const __nv_bfloat16* const bias2 = args.epi.bias2;
     const float* const colvec = args.epi.colvec;
     const __nv_bfloat16* const residual = args.epi.residual;
-    const int ld_res = args.epi.ld_res, ld_out = args.epi.ld_out, f16_begin = args.epi.f16_begin;
+    const int ld_res = args.epi.ld_res, ld_out = args.epi.ld_out;
     const bool geglu = args.epi.mode == GEMM_GEGLU;
     __nv_bfloat16* const out = args.epi.out;
     const bool has_cols = partial == nullptr && (bias || bias2 || colvec);
@@ -481,14 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
         __nv_bfloat16* dst = out + grow * ld_out + nb;
-        if (full && f16_begin > 0 && nb >= f16_begin) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            d4[w] = make_uint4(pack_f16x2(v[8 * w + 0], v[8 * w + 1]), pack_f16x2(v[8 * w + 2], v[8 * w + 3]),
-                               pack_f16x2(v[8 * w + 4], v[8 * w + 5]), pack_f16x2(v[8 * w + 6], v[8 * w + 7]));
-          }
-        } else if (full) {
+        if (full) {
           uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
@@ -577,11 +580,6 @@ __device__ __forceinline__ void splitk_reduce_vec(const float* __restrict__ part
     const uint4 r = *reinterpret_cast<const uint4*>(epi.residual + (size_t)row * epi.ld_res + c);
     v[0] += bf16lo(r.x); v[1] += bf16hi(r.x); v[2] += bf16lo(r.y); v[3] += bf16hi(r.y);
     v[4] += bf16lo(r.z); v[5] += bf16hi(r.z); v[6] += bf16lo(r.w); v[7] += bf16hi(r.w);
-  }
-  if (epi.f16_begin > 0 && c >= epi.f16_begin) {
-    *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) =
-        make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
-    return;
   }
   const uint4 o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                              pack_bf16x2(v[6], v[7]));
@@ -951,6 +949,7 @@ int gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   args.epi = p.epi;
   args.partial = g.splits > 1 ? p.splitk_ws : nullptr;
   args.err = p.err;
+  args.hold_spins = p.hold_spins;
   const int bn = g.bn;
 
   GemmMaps maps;

@@ -47,7 +47,6 @@ struct GemmEpi {
   __nv_bfloat16* out;             // [M][ld_out]
   int32_t ld_out;
   int32_t mode;                   // GemmMode
-  int32_t f16_begin;              // > 0: output columns >= f16_begin are stored as FP16 (a multiple of 32)
   // Row statistics for a LayerNorm folded into the next GEMM. rowstat_out: each
   // output row's sum and sum of squares of the stored BF16 values are added into
   // rowstat_out[2*row .. 2*row+1] as 64-bit fixed point (scales 2^24 and 2^18);
@@ -87,6 +86,10 @@ struct GemmProblem {
   int32_t force_splits;  // 0 = heuristic, 1 = no split
   float* splitk_ws;      // FP32 partials [splits][Ho*Wo][N], or null
   size_t splitk_ws_bytes;
+  // > 0 (tests only): one thread of every CTA first waits on a barrier nothing
+  // completes, for at most hold_spins polls; the wait gives up and the CTA
+  // skips all its work (see sd_debug_inject_timeout)
+  int32_t hold_spins;
 };
 
 // Number of kernels gemm_tc_launch will enqueue for p (1, or 2 with split-K).

@@ -17,7 +17,8 @@ int launch_groupnorm(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, i
 int launch_sinusoid(float t, int proj_dim, float* out, cudaStream_t st);
 
 // Grouped GEMV: for each job, y[r] = act_out(sum_k W[r][k] * act_in(x[k]) + b[r]),
-// W BF16 [rows][K] row-major, x FP32 [K] shared by all jobs.
+// W BF16 [rows][K] row-major, x FP32 [K] shared by all jobs; with accum_out the
+// result is added to y[r] instead of replacing it.
 constexpr int kMaxGemvJobs = 32;
 struct GemvJob {
   const __nv_bfloat16* W;
@@ -26,11 +27,20 @@ struct GemvJob {
   int32_t rows;
 };
 struct GemvBatch {
-  int32_t njobs, K, silu_in, silu_out;
+  int32_t njobs, K, silu_in, silu_out, accum_out;
   const float* x;
   GemvJob job[kMaxGemvJobs];
 };
 int launch_gemv(const GemvBatch& batch, cudaStream_t st);
+
+// SDXL added-conditioning input: out = [text (BF16 -> FP32) | phi(ids[0]) | ... ],
+// phi(v) = [cos(v f_i) | sin(v f_i)] of width dim, f_i = 10000^(-i/(dim/2)).
+constexpr int kMaxAddIds = 8;
+struct AddIds {
+  float v[kMaxAddIds];
+};
+int launch_add_embed_input(const __nv_bfloat16* text, int text_dim, const AddIds& ids, int n_ids, int dim,
+                           float* out, cudaStream_t st);
 
 // Nearest 2x upsample of NHWC [H, W, C] into [2H, 2W, C].
 int launch_upsample2x(const __nv_bfloat16* x, int H, int W, int C, __nv_bfloat16* y, cudaStream_t st);

@@ -56,7 +56,8 @@ __global__ void gemv_kernel(const __grid_constant__ GemvBatch batch) {
   for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) {
     if (job.b) acc += __bfloat162float(job.b[row]);
-    job.y[row] = batch.silu_out ? silu_f(acc) : acc;
+    const float r = batch.silu_out ? silu_f(acc) : acc;
+    job.y[row] = batch.accum_out ? job.y[row] + r : r;
   }
 }
 
@@ -67,6 +68,36 @@ int launch_gemv(const GemvBatch& batch, cudaStream_t st) {
   const int blocks = (int)((rows + warps - 1) / warps);
   if (blocks == 0) return 0;
   return (int)launch_pdl(gemv_kernel, dim3(blocks), dim3(warps * 32), batch.K * sizeof(float), st, batch);
+}
+
+// SDXL added conditioning (tutorial page, SDXL conditioning paragraphs): the
+// pooled text vector, then each size/crop scalar Fourier-encoded like the
+// timestep, in FP32 for the first linear layer.
+__global__ void add_embed_input_kernel(const __nv_bfloat16* __restrict__ text, int text_dim, AddIds ids, int n_ids,
+                                       int dim, float* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  const int half = dim / 2;
+  const int total = text_dim + n_ids * dim;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    if (i < text_dim) {
+      out[i] = __bfloat162float(text[i]);
+      continue;
+    }
+    const int j = (i - text_dim) / dim;
+    const int k = (i - text_dim) % dim;
+    const int fi = k < half ? k : k - half;
+    const double f = exp(-9.210340371976184 * (double)fi / (double)half);  // ln(10000)
+    const double a = (double)ids.v[j] * f;
+    out[i] = (float)(k < half ? cos(a) : sin(a));
+  }
+}
+
+int launch_add_embed_input(const __nv_bfloat16* text, int text_dim, const AddIds& ids, int n_ids, int dim,
+                           float* out, cudaStream_t st) {
+  const int total = text_dim + n_ids * dim;
+  return (int)launch_pdl(add_embed_input_kernel, dim3((total + 255) / 256), dim3(256), 0, st, text, text_dim, ids,
+                         n_ids, dim, out);
 }
 
 // Nearest 2x (UpSample bullet): y[i][j] = x[i/2][j/2], one 16-byte vector per thread.

@@ -16,45 +16,31 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
-#include <mutex>
-
 #include "kernels.cuh"
+#include "profile.h"
 #include "sd_api.h"
+#include "weights.h"
 
 namespace {
 
 constexpr int kNoAllocMaxDim = 4096;
-constexpr int kMaxDevices = 64;
 
 // File-scope scratch: [0, kNoAllocMaxDim) = phi(t), [kNoAllocMaxDim, 2*kNoAllocMaxDim) = hidden.
 static __device__ __align__(256) float g_time_scratch[2 * kNoAllocMaxDim];
 
-std::mutex g_mu;
-float* g_scratch_ptr[kMaxDevices];
-
 // Device address of g_time_scratch on the current device. In host code the
-// symbol name is only a host-side stand-in, so the address is looked up once per
-// device with that device current.
+// symbol name is only a host-side stand-in, so the address is asked for with
+// the device current, on every call: the query is a host call that allocates
+// nothing, and a fresh answer stays right after a device reset reloads the module.
 sd_status scratch_ptr(float** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SD_ERR_LAUNCH;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_time_scratch) != cudaSuccess || !p) {
-      (void)cudaGetLastError();
-      return SD_ERR_LAUNCH;
-    }
-    g_scratch_ptr[dev] = static_cast<float*>(p);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_time_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();
+    return SD_ERR_LAUNCH;
   }
-  *out = g_scratch_ptr[dev];
+  *out = static_cast<float*>(p);
   return SD_OK;
 }
-
-// Byte offsets of the four tensors in the packed time-MLP buffer: each tensor
-// starts on a 256-byte boundary, in table order (lin1.weight, lin1.bias,
-// lin2.weight, lin2.bias).
-inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
 }  // namespace
 
@@ -80,13 +66,16 @@ extern "C" sd_status sd_time_embed_noalloc(const sd_time_cfg* cfg, const void* p
 
   const int P = cfg->proj_dim, T = cfg->temb_dim;
   const uint8_t* base = static_cast<const uint8_t*>(packed_w);
-  const int64_t l1w = 0;
-  const int64_t l1b = align256(l1w + (int64_t)T * P * 2);
-  const int64_t l2w = align256(l1b + (int64_t)T * 2);
-  const int64_t l2b = align256(l2w + (int64_t)T * T * 2);
+  // packed offsets from the same weight table sd_time_embed uses (host only)
+  sdw::Table tab;
+  const sdw::TimeW tw = sdw::add_time(tab, "time", P, T);
+  const int64_t l1w = tw.l1w, l1b = tw.l1b, l2w = tw.l2w, l2b = tw.l2b;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  if (sdk::launch_sinusoid(timestep, P, phi, st) != 0) return SD_ERR_LAUNCH;
+  {
+    sdp::Scope sc("sinusoid", sdp::F_OTHER, 0, 4.0 * P, st);
+    if (sdk::launch_sinusoid(timestep, P, phi, st) != 0) return SD_ERR_LAUNCH;
+  }
   sdk::GemvBatch b;
   memset(&b, 0, sizeof(b));
   b.njobs = 1;
@@ -95,12 +84,18 @@ extern "C" sd_status sd_time_embed_noalloc(const sd_time_cfg* cfg, const void* p
   b.x = phi;
   b.job[0] = {reinterpret_cast<const __nv_bfloat16*>(base + l1w), reinterpret_cast<const __nv_bfloat16*>(base + l1b),
               hid, T};
-  if (sdk::launch_gemv(b, st) != 0) return SD_ERR_LAUNCH;
+  {
+    sdp::Scope sc("gemv", sdp::F_GEMV, 2.0 * T * P, 2.0 * T * P, st);
+    if (sdk::launch_gemv(b, st) != 0) return SD_ERR_LAUNCH;
+  }
   b.K = T;
   b.silu_out = 0;
   b.x = hid;
   b.job[0] = {reinterpret_cast<const __nv_bfloat16*>(base + l2w), reinterpret_cast<const __nv_bfloat16*>(base + l2b),
               temb_out, T};
-  if (sdk::launch_gemv(b, st) != 0) return SD_ERR_LAUNCH;
+  {
+    sdp::Scope sc("gemv", sdp::F_GEMV, 2.0 * T * T, 2.0 * T * T, st);
+    if (sdk::launch_gemv(b, st) != 0) return SD_ERR_LAUNCH;
+  }
   return SD_OK;
 }

@@ -158,6 +158,8 @@ UNetW add_unet(Table& tab, const sd_unet_cfg& cfg) {
   const int L = cfg.n_levels;
   const int* ch = cfg.block_channels;
   u.time = add_time(tab, "time", cfg.time_proj_dim, cfg.temb_dim);
+  u.has_add = cfg.add_text_dim > 0;
+  if (u.has_add) u.add = add_time(tab, "add", cfg.add_text_dim + cfg.add_time_ids * cfg.add_time_dim, cfg.temb_dim);
   u.conv_in_kp = conv_in_kp(cfg.in_channels);
   u.conv_in = add_conv_in(tab, "conv_in", cfg.in_channels, ch[0], u.conv_in_kp);
   std::vector<int> skips;

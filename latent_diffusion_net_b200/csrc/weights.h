@@ -101,6 +101,8 @@ TxW add_transformer(Table& tab, const std::string& prefix, int C, int depth, int
 // Whole U-Net: module order follows the forward pass.
 struct UNetW {
   TimeW time;
+  bool has_add;  // SDXL added conditioning MLP (same shape as the time MLP)
+  TimeW add;
   ConvW conv_in;
   int conv_in_kp;
   struct Level {

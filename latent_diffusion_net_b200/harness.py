@@ -1,4 +1,4 @@
-"""Device-side driver of the five workloads through the C ABI.
+"""Device-side driver of the synthetic workloads through the C ABI.
 
 PyTorch supplies device memory and streams only; every step of the denoiser
 runs in the library's kernels, called through ``binding``. Inputs and weights
@@ -12,7 +12,7 @@ import torch
 
 from . import binding as B
 from . import synth
-from .workloads import CTX_LEN, TIMESTEP, WORKLOADS
+from .workloads import CTX_LEN, SDXL_TIME_IDS, TIMESTEP, UNETS, WORKLOADS
 
 
 def to_dev_bf16(a: np.ndarray, device="cuda") -> torch.Tensor:
@@ -103,7 +103,9 @@ class Workload:
     """Builds the modules, weights and inputs of workload ``wid`` on the device
     and runs one step through the ABI."""
 
-    def __init__(self, wid, device="cuda", affine_noise=False):
+    def __init__(self, wid, device="cuda", affine_noise=False, canonical=None):
+        """``canonical``: already generated canonical buffers of this workload's
+        modules (the same seed and tables), to skip drawing them again."""
         self.wid = wid
         self.spec = dict(WORKLOADS[wid])
         self.device = device
@@ -111,7 +113,7 @@ class Workload:
         seed = s["seed"]
         self.modules = []
         if s["kind"] == "unet":
-            self.cfg = B.unet_cfg(height=s["H"], width=s["W"], ctx_dim=s["ctx_dim"])
+            self.cfg = B.unet_cfg(height=s["H"], width=s["W"], **UNETS[s["unet"]])
             self.modules = [Module("unet", self.cfg)]
         else:
             self.modules.append(Module("time", B.time_cfg()))
@@ -125,7 +127,7 @@ class Workload:
             if s["kind"] == "stage4":
                 hw = s["inpaint_hw"]
                 self.modules.append(Module("conv", B.conv_cfg(hw, hw, 9, 320), B.SD_CONV_IN))
-        self.canonical = generate_canonical(self.modules, seed, affine_noise)
+        self.canonical = canonical if canonical is not None else generate_canonical(self.modules, seed, affine_noise)
         for m, c in zip(self.modules, self.canonical):
             m.load(c, device)
         self.inputs = make_inputs(wid)
@@ -156,7 +158,11 @@ class Workload:
         ctx = self.dev_inputs["ctx"] if context is None else context
         if s["kind"] == "unet":
             m = self.modules[0]
-            B.sd_unet_step(self.cfg, m.packed_dev, x, TIMESTEP, ctx, self.out, m.ws, m.ws_bytes, stream)
+            if self.cfg.add_text_dim:
+                B.sd_unet_step_cond(self.cfg, m.packed_dev, x, TIMESTEP, ctx, self.dev_inputs["text"], SDXL_TIME_IDS,
+                                    self.out, m.ws, m.ws_bytes, stream)
+            else:
+                B.sd_unet_step(self.cfg, m.packed_dev, x, TIMESTEP, ctx, self.out, m.ws, m.ws_bytes, stream)
             return self.out
         tm = self.modules[0]
         B.sd_time_embed(tm.cfg, tm.packed_dev, TIMESTEP, self.temb, tm.ws, tm.ws_bytes, stream)
@@ -183,7 +189,14 @@ def make_inputs(wid):
     s = WORKLOADS[wid]
     seed = s["seed"]
     out = {}
-    if s["kind"] == "unet":
+    if s["kind"] == "unet" and UNETS[s["unet"]]["in_channels"] == 9:
+        H, W = s["H"], s["W"]
+        noisy = synth.normal_bf16(seed, synth.IDX_NOISY, (H, W, 4))
+        masked = synth.normal_bf16(seed, synth.IDX_MASKED, (H, W, 4))
+        mask = synth.mask_rectangle(seed, H, W)[0].reshape(H, W, 1)
+        out["x"] = np.concatenate([noisy, masked, mask], axis=2)
+        out["text"] = synth.normal_bf16(seed, synth.IDX_TEXT, (UNETS[s["unet"]]["add_text_dim"],))
+    elif s["kind"] == "unet":
         out["x"] = synth.normal_bf16(seed, synth.IDX_X, (s["H"], s["W"], 4))
     else:
         out["x"] = synth.normal_bf16(seed, synth.IDX_X, (s["H"], s["W"], s["C"]))
@@ -228,36 +241,59 @@ def flops(wid):
         hw = s["H"] * s["W"]
         C = s["C"]
         return tm + res(hw, C, C) + tx(hw, C, s["depth"], s["ctx_dim"]) + conv(s["inpaint_hw"] ** 2, 9, 320)
-    # whole U-Net
-    ch = (320, 640, 1280, 1280)
-    att = (1, 1, 1, 0)
-    H = s["H"]
-    f = tm + conv(H * H, 4, 320)
-    hw = H * H
-    c_prev = 320
-    skips = [320]
-    for l in range(4):
-        for _ in range(2):
-            f += res(hw, c_prev, ch[l])
-            c_prev = ch[l]
-            if att[l]:
-                f += tx(hw, ch[l], 1, s["ctx_dim"])
-            skips.append(ch[l])
-        if l < 3:
-            f += conv(hw // 4, ch[l], ch[l])
+    return unet_flops(s["H"], s["W"], **UNETS[s["unet"]])
+
+
+def unet_flops(H, W, in_channels, block_channels, attn_depth, mid_depth, ctx_dim, add_text_dim=0, add_time_ids=0,
+               add_time_dim=256, layers_per_block=2, temb_dim=1280, proj_dim=320):
+    """Algorithmic FLOPs of one denoiser step of the given shape."""
+    def conv(hw, ci, co, k=3):
+        return 2.0 * hw * co * ci * k * k
+
+    def res(hw, ci, co):
+        f = conv(hw, ci, co) + conv(hw, co, co)
+        if ci != co:
+            f += conv(hw, ci, co, 1)
+        return f + 2.0 * temb_dim * co
+
+    def tx(hw, C, depth):
+        f = 2 * (2.0 * hw * C * C)
+        per = 2.0 * hw * C * 3 * C + 4.0 * hw * hw * C + 2.0 * hw * C * C
+        per += 2.0 * hw * C * C + 2.0 * CTX_LEN * ctx_dim * 2 * C + 4.0 * hw * CTX_LEN * C + 2.0 * hw * C * C
+        per += 2.0 * hw * C * 8 * C + 2.0 * hw * 4 * C * C
+        return f + depth * per
+
+    ch = block_channels
+    L = len(ch)
+    f = 2.0 * (proj_dim * temb_dim + temb_dim * temb_dim)
+    if add_text_dim:
+        f += 2.0 * ((add_text_dim + add_time_ids * add_time_dim) * temb_dim + temb_dim * temb_dim)
+    hw = H * W
+    f += conv(hw, in_channels, ch[0])
+    c_prev = ch[0]
+    skips = [ch[0]]
+    for lvl in range(L):
+        for _ in range(layers_per_block):
+            f += res(hw, c_prev, ch[lvl])
+            c_prev = ch[lvl]
+            if attn_depth[lvl]:
+                f += tx(hw, ch[lvl], attn_depth[lvl])
+            skips.append(ch[lvl])
+        if lvl < L - 1:
+            f += conv(hw // 4, ch[lvl], ch[lvl])
             hw //= 4
-            skips.append(ch[l])
-    f += 2 * res(hw, 1280, 1280) + tx(hw, 1280, 1, s["ctx_dim"])
-    for up in range(4):
-        l = 3 - up
-        for _ in range(3):
+            skips.append(ch[lvl])
+    f += 2 * res(hw, ch[-1], ch[-1]) + tx(hw, ch[-1], mid_depth)
+    for up in range(L):
+        lvl = L - 1 - up
+        for _ in range(layers_per_block + 1):
             cs = skips.pop()
-            f += res(hw, c_prev + cs, ch[l])
-            c_prev = ch[l]
-            if att[l]:
-                f += tx(hw, ch[l], 1, s["ctx_dim"])
-        if up < 3:
+            f += res(hw, c_prev + cs, ch[lvl])
+            c_prev = ch[lvl]
+            if attn_depth[lvl]:
+                f += tx(hw, ch[lvl], attn_depth[lvl])
+        if up < L - 1:
             hw *= 4
-            f += conv(hw, ch[l], ch[l])
-    f += conv(hw, 320, 4)
+            f += conv(hw, ch[lvl], ch[lvl])
+    f += conv(hw, ch[0], 4)
     return f

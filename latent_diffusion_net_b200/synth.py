@@ -39,6 +39,8 @@ IDX_CTX = 1        # text context
 IDX_NOISY = 2      # inpaint: noisy latent
 IDX_MASKED = 3     # inpaint: masked latent
 IDX_MASK = 4       # inpaint: mask rectangle draws
+IDX_TEXT = 5       # SDXL: pooled text embedding
+IDX_NOISE = 6      # sampler: the noise z of each reverse step (one stream, step-major)
 
 
 def stream_seed(seed: int, k: int) -> np.uint64:

@@ -17,6 +17,15 @@ timestep is 500. Activations are NHWC.
    rectangle mask; seed 3.
 5. sd21_base_unet_step_96: the whole SD2.1-base-shaped denoiser step on a 96x96
    latent with 4 channels, context [77, 1024]; seed 4.
+6. sdxl_inpaint_unet_step_128: the whole SDXL-Inpainting-shaped denoiser step on
+   a 128x128 latent: 9 input channels assembled from a noisy latent, a masked
+   latent and a rectangle mask; 3 levels (320 without attention, 640 with depth-2
+   and 1280 with depth-10 transformers), mid depth 10, context [77, 2048], and
+   the added conditioning: a pooled text vector [1280] ~ N(0, 1) and the six
+   size/crop values (1024, 1024, 0, 0, 1024, 1024); seed 5.
+7. sd21_base_unet_step_64 and 8. sd21_base_unet_step_128: the SD2.1-base step of
+   workload 5 (same weights, seed 4) on 64x64 and 128x128 latents: 4096 and 16384
+   self-attention tokens at the first level.
 """
 
 WORKLOADS = {
@@ -25,7 +34,20 @@ WORKLOADS = {
     3: dict(name="sdxl_level1_stage_640x64", seed=2, kind="stage3", H=64, W=64, C=640, depth=2, ctx_dim=2048),
     4: dict(name="sdxl_level2_stage_1280x32", seed=3, kind="stage4", H=32, W=32, C=1280, depth=10, ctx_dim=2048,
             inpaint_hw=128),
-    5: dict(name="sd21_base_unet_step_96", seed=4, kind="unet", H=96, W=96, ctx_dim=1024),
+    5: dict(name="sd21_base_unet_step_96", seed=4, kind="unet", H=96, W=96, ctx_dim=1024, unet="sd21"),
+    6: dict(name="sdxl_inpaint_unet_step_128", seed=5, kind="unet", H=128, W=128, ctx_dim=2048, unet="sdxl_inpaint"),
+    7: dict(name="sd21_base_unet_step_64", seed=4, kind="unet", H=64, W=64, ctx_dim=1024, unet="sd21"),
+    8: dict(name="sd21_base_unet_step_128", seed=4, kind="unet", H=128, W=128, ctx_dim=1024, unet="sd21"),
 }
+
+# U-Net shapes (SD2.1 architecture page section 3; SDXL-Inpainting architecture
+# page section 3; the SDXL added conditioning of the tutorial page).
+UNETS = {
+    "sd21": dict(in_channels=4, block_channels=(320, 640, 1280, 1280), attn_depth=(1, 1, 1, 0), mid_depth=1,
+                 ctx_dim=1024, add_text_dim=0, add_time_ids=0),
+    "sdxl_inpaint": dict(in_channels=9, block_channels=(320, 640, 1280), attn_depth=(0, 2, 10), mid_depth=10,
+                         ctx_dim=2048, add_text_dim=1280, add_time_ids=6),
+}
+SDXL_TIME_IDS = (1024.0, 1024.0, 0.0, 0.0, 1024.0, 1024.0)  # original size, crop top-left, target size
 TIMESTEP = 500.0
 CTX_LEN = 77

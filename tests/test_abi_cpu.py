@@ -49,8 +49,7 @@ def oracle_rows(table, prefix):
 
 @pytest.mark.parametrize("cfg", [model.SD21_BASE, model.SDXL_INPAINT])
 def test_unet_table_matches_oracle(cfg):
-    c = B.unet_cfg(in_channels=cfg.in_channels, block_channels=cfg.block_channels, attn_depth=cfg.attn_depth,
-                   mid_depth=cfg.mid_depth, ctx_dim=cfg.ctx_dim, height=96, width=96)
+    c = B.unet_cfg_from(cfg, 96, 96)
     rows, canon, packed = B.sd_unet_weight_layout(c)
     ora = model.enumerate_unet_params(cfg)
     assert strip(rows, "") == oracle_rows(ora, "")
@@ -192,3 +191,39 @@ def test_gemm_override_validation():
             B.sd_gemm_override(bn, sp)
     for bn, sp in [(32, 1), (256, 16), (160, 0), (0, 0)]:
         B.sd_gemm_override(bn, sp)
+
+
+def test_conditioned_step_and_hooks_validate_on_host():
+    """SDXL added conditioning is checked before any launch; the record and
+    timeout-injection hooks reject bad arguments."""
+    fake = 1 << 20
+    sdxl = B.unet_cfg_from(model.SDXL_INPAINT, 128, 128)
+    assert B.sd_unet_workspace_size(sdxl) > B.sd_unet_workspace_size(B.unet_cfg(height=128, width=128,
+                                                                                   in_channels=9,
+                                                                                   block_channels=(320, 640, 1280),
+                                                                                   attn_depth=(0, 2, 10),
+                                                                                   mid_depth=10, ctx_dim=2048))
+    # the plain step cannot serve a config with added conditioning
+    assert B.sd_unet_step(sdxl, fake, fake, 500.0, fake, fake, fake, 10 ** 11, check=False) == 1
+    assert B.sd_unet_step_cond(sdxl, fake, fake, 500.0, fake, None, [1024.0] * 6, fake, fake, 10 ** 11,
+                               check=False) == 1
+    assert B.sd_unet_step_cond(sdxl, fake, fake, 500.0, fake, fake, None, fake, fake, 10 ** 11, check=False) == 1
+    assert B.sd_unet_step_cond(sdxl, fake, fake, 500.0, fake, fake + 4, [0.0] * 6, fake, fake, 10 ** 11,
+                               check=False) == 4
+    bad = B.unet_cfg_from(model.SDXL_INPAINT, 128, 128)
+    bad.add_time_ids = 9
+    assert B.sd_unet_step_cond(bad, fake, fake, 500.0, fake, fake, [0.0] * 9, fake, fake, 10 ** 11,
+                               check=False) == 3
+    bad = B.unet_cfg_from(model.SDXL_INPAINT, 128, 128)
+    bad.add_time_dim = 255
+    assert B.sd_unet_step_cond(bad, fake, fake, 500.0, fake, fake, [0.0] * 6, fake, fake, 10 ** 11,
+                               check=False) == 2
+    for n, spins in [(-1, 10), (1, 0), (1, (1 << 24) + 1)]:
+        with pytest.raises(RuntimeError):
+            B.sd_debug_inject_timeout(n, spins)
+    B.sd_debug_inject_timeout(0, 0)
+    with pytest.raises(RuntimeError):
+        B.sd_record_begin(fake + 8, 1024)
+    B.sd_record_begin(fake, 0)
+    assert B.sd_record_end() == (0, 0)
+    assert B.sd_record_read() == []

@@ -8,7 +8,7 @@ the bound per operator is 1e-2 and per block 2e-2."""
 import numpy as np
 import pytest
 
-from gpu_util import chw, dev_np, hwc, oracle_params, rel_l2
+from gpu_util import assert_close, chw, dev_np, hwc, oracle_params
 from oracle import model
 import oracle
 from latent_diffusion_net_b200 import synth
@@ -40,7 +40,7 @@ def test_time_embed():
     B.sd_time_embed(m.cfg, m.packed_dev, 500.0, temb, m.ws, m.ws_bytes)
     torch.cuda.synchronize()
     ref = oracle.time_mlp(p, 500.0)
-    assert rel_l2(temb.cpu().numpy(), ref) < 1e-4
+    assert_close(temb.cpu().numpy(), ref, 1e-4)
     assert B.sd_query_device_status(m.ws) == 0
 
 
@@ -61,7 +61,7 @@ def test_conv_in(hw, cin):
                       y, m.ws, m.ws_bytes)
     torch.cuda.synchronize()
     ref = hwc(oracle.conv_in(chw(x), p))
-    assert rel_l2(dev_np(y, (hw, hw, 320)), ref) < OP_TOL
+    assert_close(dev_np(y, (hw, hw, 320)), ref, OP_TOL)
 
 
 @pytest.mark.parametrize("H,W,C", [(8, 8, 64), (12, 12, 320), (6, 10, 128)])
@@ -73,7 +73,7 @@ def test_upsample_conv(H, W, C):
     B.sd_conv_fwd(m.cfg, B.SD_CONV_UPSAMPLE, m.packed_dev, Hn.to_dev_bf16(x), None, None, y, m.ws, m.ws_bytes)
     torch.cuda.synchronize()
     ref = hwc(oracle.upsample(chw(x), p, "up"))
-    assert rel_l2(dev_np(y, (2 * H, 2 * W, C)), ref) < OP_TOL
+    assert_close(dev_np(y, (2 * H, 2 * W, C)), ref, OP_TOL)
 
 
 @pytest.mark.parametrize("H,W,C", [(24, 24, 320), (16, 10, 128), (64, 64, 640)])
@@ -85,7 +85,7 @@ def test_downsample_conv(H, W, C):
     B.sd_conv_fwd(m.cfg, B.SD_CONV_DOWNSAMPLE, m.packed_dev, Hn.to_dev_bf16(x), None, None, y, m.ws, m.ws_bytes)
     torch.cuda.synchronize()
     ref = hwc(oracle.downsample(chw(x), p, "down"))
-    assert rel_l2(dev_np(y, (H // 2, W // 2, C)), ref) < OP_TOL
+    assert_close(dev_np(y, (H // 2, W // 2, C)), ref, OP_TOL)
 
 
 @pytest.mark.parametrize("H,W,C", [(20, 20, 320), (96, 96, 320)])
@@ -99,7 +99,7 @@ def test_output_head(H, W, C):
     torch.cuda.synchronize()
     g = oracle.silu(oracle.group_norm(chw(x), p["out.norm.gamma"], p["out.norm.beta"], 32, 1e-5))
     ref = hwc(oracle.conv2d(g, p["conv_out.weight"], p["conv_out.bias"], 1, 1))
-    assert rel_l2(dev_np(y, (H, W, 4)), ref) < OP_TOL
+    assert_close(dev_np(y, (H, W, 4)), ref, OP_TOL)
 
 
 RES_CASES = [
@@ -126,7 +126,7 @@ def test_resblock(H, W, cx, cs, co, affine):
     torch.cuda.synchronize()
     xin = chw(x) if not cs else np.concatenate([chw(x), chw(sk)], axis=0)
     ref = hwc(oracle.resblock(xin, temb, p, "r"))
-    assert rel_l2(dev_np(y, (H, W, co)), ref) < BLOCK_TOL
+    assert_close(dev_np(y, (H, W, co)), ref, BLOCK_TOL)
     assert B.sd_query_device_status(m.ws) == 0
 
 
@@ -153,9 +153,9 @@ def test_transformer(H, W, C, depth, D, L, affine):
     torch.cuda.synchronize()
     ref = hwc(oracle.transformer(chw(x), ctx, p, "t", depth))
     got = dev_np(y, (H, W, C))
-    assert rel_l2(got, ref) < BLOCK_TOL
+    assert_close(got, ref, BLOCK_TOL)
     # the residual path dominates the output: also check the block's own contribution
-    assert rel_l2(got - x, ref - chw(x).transpose(1, 2, 0)) < 3 * BLOCK_TOL
+    assert_close(got - x, ref - chw(x).transpose(1, 2, 0), 3 * BLOCK_TOL)
 
 
 def test_transformer_in_place():
@@ -169,7 +169,7 @@ def test_transformer_in_place():
     B.sd_transformer_fwd(cfg, m.packed_dev, xd, Hn.to_dev_bf16(ctx), xd, m.ws, m.ws_bytes)
     torch.cuda.synchronize()
     ref = hwc(oracle.transformer(chw(x), ctx, p, "t", 1))
-    assert rel_l2(dev_np(xd, (H, W, C)), ref) < BLOCK_TOL
+    assert_close(dev_np(xd, (H, W, C)), ref, BLOCK_TOL)
 
 
 def test_small_unet_step():
@@ -186,5 +186,5 @@ def test_small_unet_step():
     B.sd_unet_step(cfg, m.packed_dev, Hn.to_dev_bf16(lat), 500.0, Hn.to_dev_bf16(ctx), y, m.ws, m.ws_bytes)
     torch.cuda.synchronize()
     ref = hwc(oracle.unet_step(chw(lat), 500.0, ctx, p, cfg_o))
-    assert rel_l2(dev_np(y, (16, 16, 4)), ref) < 5e-2
+    assert_close(dev_np(y, (16, 16, 4)), ref, 5e-2)
     assert B.sd_query_device_status(m.ws) == 0

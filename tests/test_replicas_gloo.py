@@ -57,7 +57,7 @@ def test_single_rank_needs_no_process_group():
 
 def test_reference_arm_other_ranks_exit_without_work():
     class Args:
-        steps, warmup = 1, 0
+        steps, warmup, workload = 1, 0, 5
 
     assert bench.run_reference(Args, rank=1, world=2) == 0
 
@@ -72,10 +72,26 @@ def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch)
     prof = tmp_path / "profiles"
     prof.mkdir()
     digest = hashlib.sha256(src.read_bytes()).hexdigest()
-    (prof / "k_dram_traffic_unet_step_sd21_96.md").write_text(
+    (prof / "k_dram_traffic_sd21_base_unet_step_96.md").write_text(
         "summary\n\ntraffic_bytes_per_launch: 1234\nsource: kernel.cu\nsource_sha256: " + digest + "\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.measured_traffic("k") == 1234.0
+    assert bench.measured_traffic("k", "sd21_base_unet_step_96") == 1234.0
+    assert bench.measured_traffic("k", "other_workload") is None
     src.write_text("// version 2\n")
-    assert bench.measured_traffic("k") is None
-    assert bench.measured_traffic("missing") is None
+    assert bench.measured_traffic("k", "sd21_base_unet_step_96") is None
+    assert bench.measured_traffic("missing", "sd21_base_unet_step_96") is None
+
+
+def test_peak_choice_follows_region_length_and_power_cap():
+    peaks = {"bf16_tflops": 1674.6, "bf16_tflops_sustained": 1363.4, "hbm_gbs": 6547.5}
+    assert bench.choose_peak(peaks, "measured", 0.12, {"reasons": []})[0] == 1674.6
+    assert bench.choose_peak(peaks, "measured", 0.12, {"reasons": ["sw_power_cap"]})[0] == 1363.4
+    assert bench.choose_peak(peaks, "measured", 1.7, {"reasons": []})[0] == 1363.4
+
+
+def test_reference_arm_splits_one_pass_into_the_timed_steps():
+    """The reference arm's module list covers the whole step in forward order."""
+    names = bench.oracle_stage_names(5)
+    assert names[0] == "temb" and names[-1] == "out"
+    assert sum(n.endswith(".res.0") or n.endswith(".res.1") or n.endswith(".res.2") for n in names) == 22
+    assert sum(".attn." in n for n in names) == 16 and "mid.attn.0" in names
