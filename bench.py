@@ -181,7 +181,7 @@ def oracle_params_of(wid, canonical):
     from latent_diffusion_net_b200.workloads import WORKLOADS
 
     s = WORKLOADS[wid]
-    if s["kind"] == "unet":
+    if s["kind"] in ("unet", "denoise"):
         tables = [model.enumerate_unet_params(oracle_unet_cfg(wid))]
     else:
         C = s["C"]
@@ -221,6 +221,21 @@ def oracle_stages(wid, params, inputs):
     s = WORKLOADS[wid]
     x = np.ascontiguousarray(np.asarray(inputs["x"], dtype=np.float64).transpose(2, 0, 1))
     ctx = np.asarray(inputs["ctx"], dtype=np.float64)
+    if s["kind"] == "denoise":
+        # one guided DDIM iteration: the denoiser with each context, guidance, update
+        from oracle import sampler
+        cfg = oracle_unet_cfg(wid)
+        eps = []
+        for c in (ctx, np.asarray(inputs["ctx_uncond"], dtype=np.float64)):
+            out = None
+            for name, h in oracle.unet_stages(x, float(s["timestep"]), c, params, cfg):
+                out = h
+                yield name, h
+            eps.append(out)
+        betas = sampler.linear_betas()
+        t = s["timestep"]
+        yield "update", sampler.ddim_step(x, sampler.cfg_combine(eps[0], eps[1], s["guidance"]), t, t - 1, betas)
+        return
     if s["kind"] == "unet":
         cfg = oracle_unet_cfg(wid)
         kw = {"add_text": inputs["text"], "add_time_ids": SDXL_TIME_IDS} if cfg.add_embed_dim else {}
@@ -258,13 +273,19 @@ def oracle_stage_names(wid):
     """Module names of the oracle's pass over workload ``wid`` (no arithmetic)."""
     from latent_diffusion_net_b200.workloads import WORKLOADS
     s = WORKLOADS[wid]
+    if s["kind"] == "denoise":
+        one = oracle_unet_stage_names(oracle_unet_cfg(wid))
+        return one + one + ["update"]
     if s["kind"] != "unet":
         nb = 2 if s["kind"] == "stage3" else 1
         names = ["temb"] + [n for b in range(nb) for n in (f"r{b}", f"t{b}")]
         if s["kind"] in ("stage3", "stage4"):
             names.append("extra")
         return names
-    cfg = oracle_unet_cfg(wid)
+    return oracle_unet_stage_names(oracle_unet_cfg(wid))
+
+
+def oracle_unet_stage_names(cfg):
     L = len(cfg.block_channels)
     names = ["temb", "conv_in"]
     for lvl in range(L):
@@ -356,8 +377,11 @@ def aggregate_steps_per_s(ms_step, world):
 
 
 def workload_config(spec):
-    cfg = {"workload": spec["name"], "timestep": 500}
-    if spec["kind"] == "unet":
+    cfg = {"workload": spec["name"], "timestep": spec.get("timestep", 500)}
+    if spec["kind"] == "denoise":
+        cfg.update({"latent": [1, 4, spec["H"], spec["W"]], "context": [2, 77, spec["ctx_dim"]],
+                    "guidance": spec["guidance"], "sampler": "ddim, linear schedule 1e-4..0.02, T=1000"})
+    elif spec["kind"] == "unet":
         c = 9 if spec["unet"] == "sdxl_inpaint" else 4
         cfg.update({"latent": [1, c, spec["H"], spec["W"]], "context": [1, 77, spec["ctx_dim"]]})
     else:
@@ -386,7 +410,7 @@ def run_reference(args, rank, world):
     wid = args.workload
     spec = WORKLOADS[wid]
     step_flops = flops(wid)
-    if spec["kind"] == "unet":
+    if spec["kind"] in ("unet", "denoise"):
         tables = [model.enumerate_unet_params(oracle_unet_cfg(wid))]
     else:
         C = spec["C"]
@@ -622,7 +646,7 @@ def main():
     # ------------------------------------------------------------- end to end through the ABI
     host_in = {k: t.cpu().pin_memory() for k, t in wl.dev_inputs.items()}
     dev_in = {k: torch.empty_like(t) for k, t in wl.dev_inputs.items()}
-    out_h = torch.empty(wl.out.shape, dtype=torch.bfloat16).pin_memory()
+    out_h = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
     saved = dict(wl.dev_inputs)
     wl.dev_inputs.update(dev_in)
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
@@ -647,7 +671,7 @@ def main():
     e2e_ms = slowest_rank_ms(e2e_ms, world, dev)
     e2e = {"value": aggregate_steps_per_s(e2e_ms, world), "unit": UNIT,
            "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host_in.values())),
-           "d2h_bytes_per_step": out_h.numel() * 2, "ms_per_step": e2e_ms,
+           "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "ms_per_step": e2e_ms,
            "path": f"pinned host {'+'.join(host_in)} -> device, the workload's eager ABI calls, output -> "
                    "pinned host, stream synchronised every step"}
     st = B.sd_query_device_status(wl.modules[0].ws, stream)

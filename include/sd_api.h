@@ -283,6 +283,69 @@ sd_status sd_unet_step_cond(const sd_unet_cfg* cfg, const void* packed_w, const 
                             const void* context, const void* add_text, const float* add_time_ids, void* eps_out,
                             void* workspace, size_t ws_bytes, sd_stream_t stream);
 
+/* ---------------------------------------------------------------- sampling
+ * The steps either side of the denoiser [TUT, DDPM paragraphs]: the forward
+ * process q(x_t | x_{t-1}) = N(sqrt(1 - beta_t) x_{t-1}, beta_t I), alpha_t =
+ * 1 - beta_t, alpha_bar_t = prod_{s<=t} alpha_s, and the reverse step
+ *   DDPM: x_{t-1} = (x_t - beta_t / sqrt(1 - alpha_bar_t) eps) / sqrt(alpha_t) + sqrt(beta_t) z
+ * as printed there; the deterministic DDIM step (Song, Meng and Ermon 2021,
+ * eta = 0; the page names the DDIM scheduler only):
+ *   x0 = (x_t - sqrt(1 - alpha_bar_t) eps) / sqrt(alpha_bar_t),
+ *   x_prev = sqrt(alpha_bar_prev) x0 + sqrt(1 - alpha_bar_prev) eps;
+ * and classifier-free guidance (the "CFG scale" of the SD1.5 anatomy page):
+ *   eps = eps_uncond + guidance * (eps_cond - eps_uncond).
+ * Timesteps t run from 1 to T; alphas_cumprod[t - 1] is alpha_bar_t. */
+enum { SD_SCHED_LINEAR = 0, SD_SCHED_COSINE = 1 };
+enum { SD_SAMPLER_DDPM = 0, SD_SAMPLER_DDIM = 1 };
+
+/* Host only. SD_SCHED_LINEAR: beta rises linearly from beta_start to beta_end
+ * over T steps (the page: 0.0001 to 0.02, T = 1000; the DDIM scheduler's
+ * beta_start 0.00085 is another choice). SD_SCHED_COSINE: the cosine schedule
+ * of Nichol and Dhariwal (2021), named on the page, with s = 0.008 and beta
+ * clipped at 0.999 (beta_start/end unused). Writes alphas_cumprod[T]. */
+sd_status sd_schedule(int32_t kind, int32_t T, double beta_start, double beta_end, double* alphas_cumprod);
+
+/* One reverse step on a latent of n elements, in place on the FP32 state x
+ * (x_t in, x_prev out). alpha_bar_t / alpha_bar_prev: the schedule at the current
+ * and the next timestep (alpha_bar_prev = 1 after the last step; for DDPM the
+ * next timestep is t - 1, beta_t = 1 - alpha_bar_t / alpha_bar_prev).
+ * eps_cond / eps_uncond: BF16 [n] U-Net outputs; eps_uncond = NULL means no
+ * guidance. noise: FP32 [n] z of the DDPM step, NULL = none (always none for
+ * DDIM). x_bf16: NULL, or a BF16 [n / out_ch][ld] buffer whose first out_ch
+ * channels of each pixel receive the new x (the next U-Net input; the other
+ * ld - out_ch channels are left as they are). Device pointers, 16-byte aligned. */
+typedef struct {
+  int32_t kind;          /* SD_SAMPLER_* */
+  int64_t n;             /* latent elements (H * W * out_ch) */
+  int32_t out_ch;        /* channels of the latent (4) */
+  int32_t ld;            /* channels per pixel of x_bf16 (out_ch, or 9 for inpainting) */
+  float guidance;        /* classifier-free guidance scale */
+  double alpha_bar_t;
+  double alpha_bar_prev;
+} sd_sampler_cfg;
+
+sd_status sd_sampler_step(const sd_sampler_cfg* cfg, float* x, const void* eps_cond, const void* eps_uncond,
+                          const float* noise, void* x_bf16, sd_stream_t stream);
+
+/* A whole sampling loop on the device, stream-ordered (no host synchronisation,
+ * so it can be captured into one CUDA graph): for each of n_steps timesteps
+ * (host array, descending, each in 1..T), run the denoiser on the current latent
+ * with ctx_cond (and again with ctx_uncond when it is not NULL, then combine with
+ * `guidance`), then sd_sampler_step to the next timestep (0 after the last).
+ * x: device FP32 [H, W, out_channels], x_T in, x_0 out. For in_channels >
+ * out_channels (inpainting) cond_latent = device BF16 [H, W, in - out] holds the
+ * channels that follow the latent in the denoiser input (masked latent, mask);
+ * else NULL. add_text_cond / add_text_uncond / add_time_ids: the SDXL added
+ * conditioning of each pass (as in sd_unet_step_cond). noise: device FP32
+ * [n_steps][H*W*out] (DDPM), or NULL. The U-Net is called with the timestep value
+ * t. Workspace: sd_denoise_workspace_size(cfg) bytes. */
+size_t sd_denoise_workspace_size(const sd_unet_cfg* cfg);
+sd_status sd_denoise(const sd_unet_cfg* cfg, const void* packed_w, int32_t sampler_kind, const double* alphas_cumprod,
+                     int32_t T, const int32_t* timesteps, int32_t n_steps, float guidance, float* x,
+                     const void* cond_latent, const void* ctx_cond, const void* ctx_uncond, const void* add_text_cond,
+                     const void* add_text_uncond, const float* add_time_ids, const float* noise, void* workspace,
+                     size_t ws_bytes, sd_stream_t stream);
+
 /* Synchronises `stream`, then reads the device error word of `workspace`:
  * SD_OK, or SD_ERR_DEVICE_TIMEOUT when a bounded wait gave up; the word is
  * cleared afterwards. */

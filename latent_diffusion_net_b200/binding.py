@@ -64,6 +64,15 @@ class sd_unet_cfg(ctypes.Structure):
                 ("add_time_dim", c_int32)]
 
 
+class sd_sampler_cfg(ctypes.Structure):
+    _fields_ = [("kind", c_int32), ("n", c_int64), ("out_ch", c_int32), ("ld", c_int32), ("guidance", c_float),
+                ("alpha_bar_t", ctypes.c_double), ("alpha_bar_prev", ctypes.c_double)]
+
+
+SD_SCHED_LINEAR, SD_SCHED_COSINE = 0, 1
+SD_SAMPLER_DDPM, SD_SAMPLER_DDIM = 0, 1
+
+
 class sd_record_entry(ctypes.Structure):
     _fields_ = [("name", c_char * 8), ("module", c_int32), ("block", c_int32), ("offset", c_int64),
                 ("rows", c_int64), ("cols", c_int64)]
@@ -109,6 +118,11 @@ _SIGS = {
     "sd_unet_step": (c_int32, [POINTER(sd_unet_cfg), _P, _P, c_float, _P, _P, _P, c_size_t, _P]),
     "sd_unet_step_cond": (c_int32, [POINTER(sd_unet_cfg), _P, _P, c_float, _P, _P, POINTER(c_float), _P, _P,
                                     c_size_t, _P]),
+    "sd_schedule": (c_int32, [c_int32, c_int32, ctypes.c_double, ctypes.c_double, POINTER(ctypes.c_double)]),
+    "sd_sampler_step": (c_int32, [POINTER(sd_sampler_cfg), _P, _P, _P, _P, _P, _P]),
+    "sd_denoise_workspace_size": (c_size_t, [POINTER(sd_unet_cfg)]),
+    "sd_denoise": (c_int32, [POINTER(sd_unet_cfg), _P, c_int32, POINTER(ctypes.c_double), c_int32, POINTER(c_int32),
+                             c_int32, c_float, _P, _P, _P, _P, _P, _P, POINTER(c_float), _P, _P, c_size_t, _P]),
     "sd_record_begin": (c_int32, [_P, c_size_t]),
     "sd_record_end": (c_int32, [POINTER(c_int32)]),
     "sd_record_read": (c_int32, [POINTER(sd_record_entry), c_int32, POINTER(c_int32)]),
@@ -312,6 +326,43 @@ def sd_unet_step_cond(cfg, packed_w, latent, timestep, context, add_text, add_ti
     s = lib().sd_unet_step_cond(ctypes.byref(cfg), _ptr(packed_w), _ptr(latent), float(timestep), _ptr(context),
                                 _ptr(add_text), ids, _ptr(eps_out), _ptr(workspace), int(ws_bytes), _stream(stream))
     return _check(s, "sd_unet_step_cond") if check else s
+
+
+def sd_schedule(kind, T=1000, beta_start=1e-4, beta_end=0.02):
+    """alpha_bar_t for t = 1..T as a list of floats (host only)."""
+    out = (ctypes.c_double * int(T))()
+    _check(lib().sd_schedule(int(kind), int(T), float(beta_start), float(beta_end), out), "sd_schedule")
+    return list(out)
+
+
+def sampler_cfg(kind, n, alpha_bar_t, alpha_bar_prev, guidance=1.0, out_ch=4, ld=None):
+    return sd_sampler_cfg(int(kind), int(n), int(out_ch), int(out_ch if ld is None else ld), float(guidance),
+                          float(alpha_bar_t), float(alpha_bar_prev))
+
+
+def sd_sampler_step(cfg, x, eps_cond, eps_uncond=None, noise=None, x_bf16=None, stream=None, check=True):
+    s = lib().sd_sampler_step(ctypes.byref(cfg), _ptr(x), _ptr(eps_cond), _ptr(eps_uncond), _ptr(noise),
+                              _ptr(x_bf16), _stream(stream))
+    return _check(s, "sd_sampler_step") if check else s
+
+
+def sd_denoise_workspace_size(cfg):
+    return lib().sd_denoise_workspace_size(ctypes.byref(cfg))
+
+
+def sd_denoise(cfg, packed_w, kind, alphas_cumprod, timesteps, guidance, x, cond_latent, ctx_cond, ctx_uncond,
+               add_text_cond, add_text_uncond, add_time_ids, noise, workspace, ws_bytes, stream=None, check=True):
+    """alphas_cumprod, timesteps, add_time_ids: host sequences; the rest device tensors (or None)."""
+    ac = (ctypes.c_double * len(alphas_cumprod))(*[float(v) for v in alphas_cumprod])
+    ts = (c_int32 * len(timesteps))(*[int(t) for t in timesteps])
+    ids = None
+    if add_time_ids is not None:
+        ids = (c_float * max(len(add_time_ids), 1))(*[float(v) for v in add_time_ids])
+    s = lib().sd_denoise(ctypes.byref(cfg), _ptr(packed_w), int(kind), ac, len(alphas_cumprod), ts, len(timesteps),
+                         float(guidance), _ptr(x), _ptr(cond_latent), _ptr(ctx_cond), _ptr(ctx_uncond),
+                         _ptr(add_text_cond), _ptr(add_text_uncond), ids, _ptr(noise), _ptr(workspace),
+                         int(ws_bytes), _stream(stream))
+    return _check(s, "sd_denoise") if check else s
 
 
 def sd_record_begin(dev_buf, nbytes):

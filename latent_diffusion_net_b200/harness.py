@@ -112,7 +112,7 @@ class Workload:
         s = self.spec
         seed = s["seed"]
         self.modules = []
-        if s["kind"] == "unet":
+        if s["kind"] in ("unet", "denoise"):
             self.cfg = B.unet_cfg(height=s["H"], width=s["W"], **UNETS[s["unet"]])
             self.modules = [Module("unet", self.cfg)]
         else:
@@ -132,6 +132,13 @@ class Workload:
             m.load(c, device)
         self.inputs = make_inputs(wid)
         self.dev_inputs = {k: to_dev_bf16(v, device) for k, v in self.inputs.items()}
+        if s["kind"] == "denoise":
+            # the sampler's FP32 latent state, updated in place by every step
+            self.dev_inputs["x"] = torch.from_numpy(self.inputs["x"].reshape(-1).astype(np.float32)).to(device)
+            m = self.modules[0]
+            m.ws_bytes = B.sd_denoise_workspace_size(self.cfg)
+            m.ws = workspace(m.ws_bytes, device)
+            self.alphas_cumprod = B.sd_schedule(B.SD_SCHED_LINEAR, 1000, 1e-4, 0.02)
         self._alloc_outputs()
 
     def _alloc_outputs(self):
@@ -139,6 +146,9 @@ class Workload:
         d = self.device
         if s["kind"] == "unet":
             self.out = torch.empty(s["H"] * s["W"] * 4, dtype=torch.bfloat16, device=d)
+            return
+        if s["kind"] == "denoise":
+            self.out = self.dev_inputs["x"]
             return
         C, H, W = s["C"], s["H"], s["W"]
         self.temb = torch.empty(1280, dtype=torch.float32, device=d)
@@ -156,6 +166,12 @@ class Workload:
         s = self.spec
         x = self.dev_inputs["x"] if latent is None else latent
         ctx = self.dev_inputs["ctx"] if context is None else context
+        if s["kind"] == "denoise":
+            m = self.modules[0]
+            B.sd_denoise(self.cfg, m.packed_dev, B.SD_SAMPLER_DDIM, self.alphas_cumprod, [s["timestep"]],
+                         s["guidance"], x, None, ctx, self.dev_inputs["ctx_uncond"], None, None, None, None, m.ws,
+                         m.ws_bytes, stream)
+            return x
         if s["kind"] == "unet":
             m = self.modules[0]
             if self.cfg.add_text_dim:
@@ -196,11 +212,13 @@ def make_inputs(wid):
         mask = synth.mask_rectangle(seed, H, W)[0].reshape(H, W, 1)
         out["x"] = np.concatenate([noisy, masked, mask], axis=2)
         out["text"] = synth.normal_bf16(seed, synth.IDX_TEXT, (UNETS[s["unet"]]["add_text_dim"],))
-    elif s["kind"] == "unet":
+    elif s["kind"] in ("unet", "denoise"):
         out["x"] = synth.normal_bf16(seed, synth.IDX_X, (s["H"], s["W"], 4))
     else:
         out["x"] = synth.normal_bf16(seed, synth.IDX_X, (s["H"], s["W"], s["C"]))
     out["ctx"] = synth.normal_bf16(seed, synth.IDX_CTX, (CTX_LEN, s["ctx_dim"]))
+    if s["kind"] == "denoise":
+        out["ctx_uncond"] = synth.normal_bf16(seed, synth.IDX_CTX_UNCOND, (CTX_LEN, s["ctx_dim"]))
     if s["kind"] == "stage4":
         hw = s["inpaint_hw"]
         out["noisy"] = synth.normal_bf16(seed, synth.IDX_NOISY, (hw, hw, 4))
@@ -241,6 +259,8 @@ def flops(wid):
         hw = s["H"] * s["W"]
         C = s["C"]
         return tm + res(hw, C, C) + tx(hw, C, s["depth"], s["ctx_dim"]) + conv(s["inpaint_hw"] ** 2, 9, 320)
+    if s["kind"] == "denoise":
+        return 2 * unet_flops(s["H"], s["W"], **UNETS[s["unet"]])
     return unet_flops(s["H"], s["W"], **UNETS[s["unet"]])
 
 

@@ -41,6 +41,7 @@ IDX_MASKED = 3     # inpaint: masked latent
 IDX_MASK = 4       # inpaint: mask rectangle draws
 IDX_TEXT = 5       # SDXL: pooled text embedding
 IDX_NOISE = 6      # sampler: the noise z of each reverse step (one stream, step-major)
+IDX_CTX_UNCOND = 7  # sampler: the unconditional context of guidance
 
 
 def stream_seed(seed: int, k: int) -> np.uint64:

@@ -26,6 +26,11 @@ timestep is 500. Activations are NHWC.
 7. sd21_base_unet_step_64 and 8. sd21_base_unet_step_128: the SD2.1-base step of
    workload 5 (same weights, seed 4) on 64x64 and 128x128 latents: 4096 and 16384
    self-attention tokens at the first level.
+9. sd21_base_guided_ddim_step_96: one iteration of a guided sampling loop on the
+   workload-5 model and latent: the denoiser with the text context and again
+   with an unconditional context [77, 1024] ~ N(0, 1) (seed 4, stream 7), the
+   guidance combination (scale 7.5) and a DDIM update at t = 500 on the page's
+   linear schedule (0.0001 -> 0.02, 1000 steps).
 """
 
 WORKLOADS = {
@@ -38,6 +43,8 @@ WORKLOADS = {
     6: dict(name="sdxl_inpaint_unet_step_128", seed=5, kind="unet", H=128, W=128, ctx_dim=2048, unet="sdxl_inpaint"),
     7: dict(name="sd21_base_unet_step_64", seed=4, kind="unet", H=64, W=64, ctx_dim=1024, unet="sd21"),
     8: dict(name="sd21_base_unet_step_128", seed=4, kind="unet", H=128, W=128, ctx_dim=1024, unet="sd21"),
+    9: dict(name="sd21_base_guided_ddim_step_96", seed=4, kind="denoise", H=96, W=96, ctx_dim=1024, unet="sd21",
+            guidance=7.5, timestep=500),
 }
 
 # U-Net shapes (SD2.1 architecture page section 3; SDXL-Inpainting architecture

@@ -138,6 +138,8 @@ TX_CASES = [
     # 320 (head, query tile) items of 32 key tiles: the self-attention key tiles are
     # spread evenly over all CTAs and split items are merged by the second kernel
     (64, 64, 640, 1, 1024, 77, False),
+    # the largest self-attention of the resolution sweep: 16384 tokens (SD2.1 level 0 at a 128x128 latent)
+    (128, 128, 320, 1, 1024, 77, False),
 ]
 
 
