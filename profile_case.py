@@ -1,6 +1,11 @@
 """Run one block of the denoiser a few times through the C ABI, for profilers.
 
-``python -m latent_diffusion_net_b200.profile_case resblock --hw 96 --c 320``
+Blocks: ``resblock``, ``transformer``, ``upsample`` and ``downsample`` (the
+resampling convolutions), ``output`` (GroupNorm + SiLU + conv_out), ``conv_in``
+(the 9-channel inpaint entry), ``time`` (the time-embedding MLP and one batch
+of resblock time projections).
+
+``python profile_case.py resblock --hw 96 --c 320``
 runs a ResnetBlock2D (C -> C, time projection from a random embedding) on a
 seeded [hw, hw, C] input; ``transformer`` runs a Transformer2DModel (depth 1,
 77 context rows of width --ctx-dim). Each iteration is one eager call of the
@@ -13,18 +18,23 @@ time per call measured with CUDA events after the warm-up calls.
 from __future__ import annotations
 
 import argparse
+import os
+import sys
 
 import numpy as np
 import torch
 
-from . import binding as B
-from . import harness as Hn
-from . import synth
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+from latent_diffusion_net_b200 import binding as B  # noqa: E402
+from latent_diffusion_net_b200 import harness as Hn  # noqa: E402
+from latent_diffusion_net_b200 import synth  # noqa: E402
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("block", choices=["resblock", "transformer"])
+    ap.add_argument("block", choices=["resblock", "transformer", "upsample", "downsample", "output", "conv_in",
+                                      "time"])
     ap.add_argument("--hw", type=int, default=96, help="latent height = width")
     ap.add_argument("--c", type=int, default=320, help="channels")
     ap.add_argument("--ctx-dim", type=int, default=1024)
@@ -38,22 +48,50 @@ def main(argv=None):
     if a.block == "resblock":
         cfg = B.resblock_cfg(hw, hw, C, C)
         m = Hn.Module("res", cfg)
-    else:
+    elif a.block == "transformer":
         cfg = B.transformer_cfg(hw, hw, C, 1, 77, a.ctx_dim)
         m = Hn.Module("attn", cfg)
+    elif a.block == "time":
+        cfg = B.time_cfg()
+        m = Hn.Module("time", cfg)
+    else:
+        kind = {"upsample": B.SD_CONV_UPSAMPLE, "downsample": B.SD_CONV_DOWNSAMPLE, "output": B.SD_CONV_OUTPUT,
+                "conv_in": B.SD_CONV_IN}[a.block]
+        cin = 9 if a.block == "conv_in" else C
+        cout = {"output": 4, "conv_in": 320}.get(a.block, C)
+        cfg = B.conv_cfg(hw, hw, cin, cout)
+        m = Hn.Module("conv", cfg, kind)
     m.load(Hn.generate_canonical([m], a.seed)[0])
-    x = Hn.to_dev_bf16(synth.normal_bf16(a.seed, synth.IDX_X, (hw, hw, C)))
-    y = torch.empty(hw * hw * C, dtype=torch.bfloat16, device="cuda")
+    if a.block == "conv_in":
+        x = Hn.to_dev_bf16(synth.normal_bf16(a.seed, synth.IDX_NOISY, (hw, hw, 4)))
+        x1 = Hn.to_dev_bf16(synth.normal_bf16(a.seed, synth.IDX_MASKED, (hw, hw, 4)))
+        x2 = Hn.to_dev_bf16(synth.mask_rectangle(a.seed, hw, hw)[0].reshape(hw, hw, 1))
+    else:
+        x = Hn.to_dev_bf16(synth.normal_bf16(a.seed, synth.IDX_X, (hw, hw, C)))
+    out_elems = {"upsample": 4 * hw * hw * C, "downsample": hw * hw * C // 4, "output": hw * hw * 4,
+                 "conv_in": hw * hw * 320}.get(a.block, hw * hw * C)
+    y = torch.empty(out_elems, dtype=torch.bfloat16, device="cuda")
     if a.block == "resblock":
         temb = torch.from_numpy(synth.normal_bf16(a.seed, synth.IDX_CTX, (1280,)).astype(np.float32)).cuda()
 
         def call():
             B.sd_resblock_fwd(cfg, m.packed_dev, x, None, temb, y, m.ws, m.ws_bytes)
-    else:
+    elif a.block == "transformer":
         ctx = Hn.to_dev_bf16(synth.normal_bf16(a.seed, synth.IDX_CTX, (77, a.ctx_dim)))
 
         def call():
             B.sd_transformer_fwd(cfg, m.packed_dev, x, ctx, y, m.ws, m.ws_bytes)
+    elif a.block == "time":
+        temb = torch.empty(1280, dtype=torch.float32, device="cuda")
+
+        def call():
+            B.sd_time_embed(cfg, m.packed_dev, 500.0, temb, m.ws, m.ws_bytes)
+    elif a.block == "conv_in":
+        def call():
+            B.sd_conv_fwd(cfg, B.SD_CONV_IN, m.packed_dev, x, x1, x2, y, m.ws, m.ws_bytes)
+    else:
+        def call():
+            B.sd_conv_fwd(cfg, kind, m.packed_dev, x, None, None, y, m.ws, m.ws_bytes)
 
     for _ in range(a.warmup):
         call()
