@@ -26,7 +26,8 @@ from .model import (UNetConfig, SD21_BASE, SDXL_INPAINT, enumerate_unet_params,
                     enumerate_resblock_params, enumerate_transformer_params,
                     enumerate_time_mlp_params, time_mlp, resblock, transformer,
                     downsample, upsample, conv_in, unet_step, unet_stages, unet_shapes,
-                    add_embedding)
+                    add_embedding, resblock_h1, self_attention_sublayer, cross_attention_sublayer,
+                    ff_sublayer)
 from . import sampler
 
 __all__ = [n for n in dir() if not n.startswith("_")]

@@ -237,6 +237,18 @@ def add_embedding(params, text, time_ids, cfg: UNetConfig, prefix="add"):
     return h[0]
 
 
+def resblock_h1(x, temb, params, prefix, groups=32, eps=1e-5):
+    """The first half of a ResnetBlock2D: h1 = Conv1(SiLU(GN1(x))) + (W_t SiLU(temb) + b_t)
+    broadcast over H, W."""
+    x = np.asarray(x, dtype=np.float64)
+    h = conv2d(silu(group_norm(x, _w(params, f"{prefix}.norm1.gamma"), _w(params, f"{prefix}.norm1.beta"),
+                               groups, eps)),
+               _w(params, f"{prefix}.conv1.weight"), _w(params, f"{prefix}.conv1.bias"), 1, 1)
+    tp = linear(silu(np.asarray(temb, dtype=np.float64))[None, :], _w(params, f"{prefix}.temb.weight"),
+                _w(params, f"{prefix}.temb.bias"))[0]
+    return h + tp[:, None, None]
+
+
 def resblock(x, temb, params, prefix, groups=32, eps=1e-5, record=None):
     """ResnetBlock2D on x [C_in, H, W] with temb [temb_dim].
 
@@ -245,12 +257,7 @@ def resblock(x, temb, params, prefix, groups=32, eps=1e-5, record=None):
     conv; Dropout is the identity. (Section 4 of the SD2.1 page; ResNetBlock
     paragraph of the tutorial page.)"""
     x = np.asarray(x, dtype=np.float64)
-    h = conv2d(silu(group_norm(x, _w(params, f"{prefix}.norm1.gamma"), _w(params, f"{prefix}.norm1.beta"),
-                               groups, eps)),
-               _w(params, f"{prefix}.conv1.weight"), _w(params, f"{prefix}.conv1.bias"), 1, 1)
-    tp = linear(silu(np.asarray(temb, dtype=np.float64))[None, :], _w(params, f"{prefix}.temb.weight"),
-                _w(params, f"{prefix}.temb.bias"))[0]
-    h = h + tp[:, None, None]
+    h = resblock_h1(x, temb, params, prefix, groups, eps)
     if record is not None:
         record[f"{prefix}.h1"] = h
     h2 = conv2d(silu(group_norm(h, _w(params, f"{prefix}.norm2.gamma"), _w(params, f"{prefix}.norm2.beta"),
@@ -261,6 +268,31 @@ def resblock(x, temb, params, prefix, groups=32, eps=1e-5, record=None):
     else:
         s = x
     return s + h2
+
+
+def self_attention_sublayer(t, params, b, head_dim=64, ln_eps=1e-5):
+    """Out-projection of SelfAttn(LN1(t)) of BasicTransformer block ``b`` (before the residual add)."""
+    n1 = layer_norm(t, _w(params, f"{b}.ln1.gamma"), _w(params, f"{b}.ln1.beta"), ln_eps)
+    a1 = attention(linear(n1, _w(params, f"{b}.attn1.q.weight"), None),
+                   linear(n1, _w(params, f"{b}.attn1.k.weight"), None),
+                   linear(n1, _w(params, f"{b}.attn1.v.weight"), None), head_dim)
+    return linear(a1, _w(params, f"{b}.attn1.out.weight"), _w(params, f"{b}.attn1.out.bias"))
+
+
+def cross_attention_sublayer(t, ctx, params, b, head_dim=64, ln_eps=1e-5):
+    """Out-projection of CrossAttn(LN2(t), ctx) of block ``b`` (before the residual add)."""
+    n2 = layer_norm(t, _w(params, f"{b}.ln2.gamma"), _w(params, f"{b}.ln2.beta"), ln_eps)
+    a2 = attention(linear(n2, _w(params, f"{b}.attn2.q.weight"), None),
+                   linear(ctx, _w(params, f"{b}.attn2.k.weight"), None),
+                   linear(ctx, _w(params, f"{b}.attn2.v.weight"), None), head_dim)
+    return linear(a2, _w(params, f"{b}.attn2.out.weight"), _w(params, f"{b}.attn2.out.bias"))
+
+
+def ff_sublayer(t, params, b, ln_eps=1e-5):
+    """GEGLU feed-forward of LN3(t) of block ``b`` (before the residual add)."""
+    n3 = layer_norm(t, _w(params, f"{b}.ln3.gamma"), _w(params, f"{b}.ln3.beta"), ln_eps)
+    return geglu_ff(n3, _w(params, f"{b}.ff.w1.weight"), _w(params, f"{b}.ff.w1.bias"),
+                    _w(params, f"{b}.ff.w2.weight"), _w(params, f"{b}.ff.w2.bias"))
 
 
 def transformer(x, ctx, params, prefix, depth, head_dim=64, groups=32, gn_eps=1e-5, ln_eps=1e-5,
@@ -277,21 +309,11 @@ def transformer(x, ctx, params, prefix, depth, head_dim=64, groups=32, gn_eps=1e
     t = linear(g.reshape(C, H * W).T, _w(params, f"{prefix}.proj_in.weight"), _w(params, f"{prefix}.proj_in.bias"))
     for d in range(depth):
         b = f"{prefix}.blocks.{d}"
-        n1 = layer_norm(t, _w(params, f"{b}.ln1.gamma"), _w(params, f"{b}.ln1.beta"), ln_eps)
-        a1 = attention(linear(n1, _w(params, f"{b}.attn1.q.weight"), None),
-                       linear(n1, _w(params, f"{b}.attn1.k.weight"), None),
-                       linear(n1, _w(params, f"{b}.attn1.v.weight"), None), head_dim)
-        o1 = linear(a1, _w(params, f"{b}.attn1.out.weight"), _w(params, f"{b}.attn1.out.bias"))
+        o1 = self_attention_sublayer(t, params, b, head_dim, ln_eps)
         t = t + o1
-        n2 = layer_norm(t, _w(params, f"{b}.ln2.gamma"), _w(params, f"{b}.ln2.beta"), ln_eps)
-        a2 = attention(linear(n2, _w(params, f"{b}.attn2.q.weight"), None),
-                       linear(ctx, _w(params, f"{b}.attn2.k.weight"), None),
-                       linear(ctx, _w(params, f"{b}.attn2.v.weight"), None), head_dim)
-        o2 = linear(a2, _w(params, f"{b}.attn2.out.weight"), _w(params, f"{b}.attn2.out.bias"))
+        o2 = cross_attention_sublayer(t, ctx, params, b, head_dim, ln_eps)
         t = t + o2
-        n3 = layer_norm(t, _w(params, f"{b}.ln3.gamma"), _w(params, f"{b}.ln3.beta"), ln_eps)
-        f = geglu_ff(n3, _w(params, f"{b}.ff.w1.weight"), _w(params, f"{b}.ff.w1.bias"),
-                     _w(params, f"{b}.ff.w2.weight"), _w(params, f"{b}.ff.w2.bias"))
+        f = ff_sublayer(t, params, b, ln_eps)
         t = t + f
         if record is not None:
             record[f"{b}.attn1"] = o1
