@@ -12,7 +12,8 @@ no code with the CUDA path. Library primitives (``numpy.tensordot``, ``@``,
 reordered beyond the definitions.
 
 ``sampler`` holds the noise schedules, the DDPM / DDIM reverse updates and
-classifier-free guidance that sit on either side of the denoiser step.
+classifier-free guidance that sit on either side of the denoiser step; ``vae``
+holds the VAE decoder that turns the denoised latent into pixels.
 
 Parity pins: see ``tests/test_oracle_*.py``. Every function here is pinned by
 at least one check that does not retype its own formula (brute-force loops,
@@ -29,5 +30,6 @@ from .model import (UNetConfig, SD21_BASE, SDXL_INPAINT, enumerate_unet_params,
                     add_embedding, resblock_h1, self_attention_sublayer, cross_attention_sublayer,
                     ff_sublayer)
 from . import sampler
+from . import vae
 
 __all__ = [n for n in dir() if not n.startswith("_")]
