@@ -183,6 +183,9 @@ def oracle_params_of(wid, canonical):
     s = WORKLOADS[wid]
     if s["kind"] in ("unet", "denoise"):
         tables = [model.enumerate_unet_params(oracle_unet_cfg(wid))]
+    elif s["kind"] == "vae":
+        from oracle import vae
+        tables = [vae.enumerate_vae_decoder_params()]
     else:
         C = s["C"]
         tables = [model.enumerate_time_mlp_params()]
@@ -220,6 +223,10 @@ def oracle_stages(wid, params, inputs):
 
     s = WORKLOADS[wid]
     x = np.ascontiguousarray(np.asarray(inputs["x"], dtype=np.float64).transpose(2, 0, 1))
+    if s["kind"] == "vae":
+        from oracle import vae
+        yield from vae.vae_stages(x, params)
+        return
     ctx = np.asarray(inputs["ctx"], dtype=np.float64)
     if s["kind"] == "denoise":
         # one guided DDIM iteration: the denoiser with each context, guidance, update
@@ -276,6 +283,11 @@ def oracle_stage_names(wid):
     if s["kind"] == "denoise":
         one = oracle_unet_stage_names(oracle_unet_cfg(wid))
         return one + one + ["update"]
+    if s["kind"] == "vae":
+        names = ["conv_in", "mid.res.0", "mid.attn", "mid.res.1"]
+        for i in range(4):
+            names += [f"up.{i}.res.{j}" for j in range(3)] + ([f"up.{i}.up"] if i < 3 else [])
+        return names + ["out"]
     if s["kind"] != "unet":
         nb = 2 if s["kind"] == "stage3" else 1
         names = ["temb"] + [n for b in range(nb) for n in (f"r{b}", f"t{b}")]
@@ -378,7 +390,9 @@ def aggregate_steps_per_s(ms_step, world):
 
 def workload_config(spec):
     cfg = {"workload": spec["name"], "timestep": spec.get("timestep", 500)}
-    if spec["kind"] == "denoise":
+    if spec["kind"] == "vae":
+        cfg.update({"latent": [1, 4, spec["H"], spec["W"]], "image": [1, 3, 8 * spec["H"], 8 * spec["W"]]})
+    elif spec["kind"] == "denoise":
         cfg.update({"latent": [1, 4, spec["H"], spec["W"]], "context": [2, 77, spec["ctx_dim"]],
                     "guidance": spec["guidance"], "sampler": "ddim, linear schedule 1e-4..0.02, T=1000"})
     elif spec["kind"] == "unet":
@@ -412,6 +426,9 @@ def run_reference(args, rank, world):
     step_flops = flops(wid)
     if spec["kind"] in ("unet", "denoise"):
         tables = [model.enumerate_unet_params(oracle_unet_cfg(wid))]
+    elif spec["kind"] == "vae":
+        from oracle import vae
+        tables = [vae.enumerate_vae_decoder_params()]
     else:
         C = spec["C"]
         tables = [model.enumerate_time_mlp_params()]

@@ -162,6 +162,28 @@ typedef struct {
   int32_t add_time_dim;       /* Fourier width per scalar (256 for SDXL), even */
 } sd_unet_cfg;
 
+/* VAE decoder [SD21 section 5; SDXLI section 5]: the denoised latent divided by
+ * scaling_factor (0.18215, [TUT]), a 1x1 post-quantisation conv, conv_in 3x3 to
+ * the widest channel count, a MidBlock (resblock, single-head self-attention
+ * over the H*W tokens, resblock), n_levels UpDecoder blocks walking
+ * block_channels backwards (512, 512, 256, 128) with layers_per_block + 1
+ * resblocks each and a nearest-2x upsampling conv after all but the last, then
+ * GroupNorm + SiLU + conv_out 3x3 to out_channels. The resblocks have no time
+ * embedding. height/width are the LATENT size; the image is 2^(n_levels-1)
+ * times larger. */
+typedef struct {
+  int32_t height;             /* latent height (96 for a 768x768 image) */
+  int32_t width;
+  int32_t latent_channels;    /* 4 */
+  int32_t out_channels;       /* 3 */
+  int32_t n_levels;           /* 4 */
+  int32_t block_channels[4];  /* 128, 256, 512, 512 (encoder order) */
+  int32_t layers_per_block;   /* 2 (each UpDecoder block has 3 resblocks) */
+  int32_t groups;             /* 32 */
+  float eps;                  /* 1e-5 */
+  float scaling_factor;       /* 0.18215 */
+} sd_vae_cfg;
+
 /* ---------------------------------------------------------------- weights (host only) */
 
 /* Enumerate the canonical tensor table. `out` may be NULL (sizes only); when
@@ -180,6 +202,8 @@ sd_status sd_transformer_weight_layout(const sd_transformer_cfg* cfg, sd_tensor_
                                        int64_t* packed_bytes);
 sd_status sd_unet_weight_layout(const sd_unet_cfg* cfg, sd_tensor_desc* out, int32_t capacity,
                                 int32_t* n_tensors, int64_t* canon_elems, int64_t* packed_bytes);
+sd_status sd_vae_weight_layout(const sd_vae_cfg* cfg, sd_tensor_desc* out, int32_t capacity, int32_t* n_tensors,
+                               int64_t* canon_elems, int64_t* packed_bytes);
 
 /* conv_kind for sd_conv_weight_layout / sd_conv_pack_weights / sd_conv_fwd. */
 enum { SD_CONV_IN = 0, SD_CONV_DOWNSAMPLE = 1, SD_CONV_UPSAMPLE = 2, SD_CONV_OUTPUT = 3 };
@@ -204,6 +228,7 @@ sd_status sd_resblock_pack_weights(const sd_resblock_cfg* cfg, const uint16_t* c
 sd_status sd_transformer_pack_weights(const sd_transformer_cfg* cfg, const uint16_t* canonical,
                                       void* packed);
 sd_status sd_unet_pack_weights(const sd_unet_cfg* cfg, const uint16_t* canonical, void* packed);
+sd_status sd_vae_pack_weights(const sd_vae_cfg* cfg, const uint16_t* canonical, void* packed);
 
 /* ---------------------------------------------------------------- workspace sizes */
 
@@ -212,6 +237,7 @@ size_t sd_conv_workspace_size(const sd_conv_cfg* cfg, int32_t conv_kind);
 size_t sd_resblock_workspace_size(const sd_resblock_cfg* cfg);
 size_t sd_transformer_workspace_size(const sd_transformer_cfg* cfg);
 size_t sd_unet_workspace_size(const sd_unet_cfg* cfg);
+size_t sd_vae_workspace_size(const sd_vae_cfg* cfg);
 
 /* ---------------------------------------------------------------- forward calls (device) */
 
@@ -346,6 +372,14 @@ sd_status sd_denoise(const sd_unet_cfg* cfg, const void* packed_w, int32_t sampl
                      const void* add_text_uncond, const float* add_time_ids, const float* noise, void* workspace,
                      size_t ws_bytes, sd_stream_t stream);
 
+/* VAE decode: latent = device BF16 [height, width, latent_channels] (NHWC),
+ * image = device BF16 [height * 2^(n_levels-1), width * 2^(n_levels-1),
+ * out_channels]. The MidBlock attention forms the full [HW, HW] score matrix in
+ * the workspace (FP32 scores, BF16 probabilities), so the workspace grows with
+ * the square of the latent's pixel count. */
+sd_status sd_vae_decode(const sd_vae_cfg* cfg, const void* packed_w, const void* latent, void* image,
+                        void* workspace, size_t ws_bytes, sd_stream_t stream);
+
 /* Synchronises `stream`, then reads the device error word of `workspace`:
  * SD_OK, or SD_ERR_DEVICE_TIMEOUT when a bounded wait gave up; the word is
  * cleared afterwards. */
@@ -402,7 +436,10 @@ sd_status sd_gemm_override(int32_t bn, int32_t splits);
  *   "h1"    conv1(SiLU(GN1(x))) + b1 + time projection of a resblock [HW, C_out];
  *   "attn1" the self-attention output after its out-projection and bias [HW, C];
  *   "attn2" the same for the cross-attention;
- *   "ff"    the GEGLU feed-forward output after its second linear and bias.
+ *   "ff"    the GEGLU feed-forward output after its second linear and bias;
+ * and the input each of them saw: "x_h1" (and "x_skip" for a concatenated
+ * skip) = the resblock input; "x_attn1", "x_attn2", "x_ff" = the residual
+ * stream entering that sublayer (before its LayerNorm).
  * These are the intermediate values of [SD21 section 4]'s block panels, for
  * comparing each sublayer with a reference. The extra outputs are computed by
  * extra launches enqueued on the call's stream (the normal outputs are
@@ -411,7 +448,7 @@ sd_status sd_gemm_override(int32_t bn, int32_t splits);
  * An entry that no longer fits is dropped and sd_record_end returns
  * SD_ERR_CAPACITY. */
 typedef struct {
-  char name[8];    /* "h1", "attn1", "attn2", "ff" */
+  char name[8];    /* "h1", "attn1", "attn2", "ff", or an input: "x_h1", "x_skip", "x_attn1", ... */
   int32_t module;
   int32_t block;
   int64_t offset;  /* byte offset in dev_buf */

@@ -64,6 +64,12 @@ class sd_unet_cfg(ctypes.Structure):
                 ("add_time_dim", c_int32)]
 
 
+class sd_vae_cfg(ctypes.Structure):
+    _fields_ = [("height", c_int32), ("width", c_int32), ("latent_channels", c_int32), ("out_channels", c_int32),
+                ("n_levels", c_int32), ("block_channels", c_int32 * 4), ("layers_per_block", c_int32),
+                ("groups", c_int32), ("eps", c_float), ("scaling_factor", c_float)]
+
+
 class sd_sampler_cfg(ctypes.Structure):
     _fields_ = [("kind", c_int32), ("n", c_int64), ("out_ch", c_int32), ("ld", c_int32), ("guidance", c_float),
                 ("alpha_bar_t", ctypes.c_double), ("alpha_bar_prev", ctypes.c_double)]
@@ -118,6 +124,11 @@ _SIGS = {
     "sd_unet_step": (c_int32, [POINTER(sd_unet_cfg), _P, _P, c_float, _P, _P, _P, c_size_t, _P]),
     "sd_unet_step_cond": (c_int32, [POINTER(sd_unet_cfg), _P, _P, c_float, _P, _P, POINTER(c_float), _P, _P,
                                     c_size_t, _P]),
+    "sd_vae_weight_layout": (c_int32, [POINTER(sd_vae_cfg), POINTER(sd_tensor_desc), c_int32, POINTER(c_int32),
+                                       POINTER(c_int64), POINTER(c_int64)]),
+    "sd_vae_pack_weights": (c_int32, [POINTER(sd_vae_cfg), POINTER(c_uint16), _P]),
+    "sd_vae_workspace_size": (c_size_t, [POINTER(sd_vae_cfg)]),
+    "sd_vae_decode": (c_int32, [POINTER(sd_vae_cfg), _P, _P, _P, _P, c_size_t, _P]),
     "sd_schedule": (c_int32, [c_int32, c_int32, ctypes.c_double, ctypes.c_double, POINTER(ctypes.c_double)]),
     "sd_sampler_step": (c_int32, [POINTER(sd_sampler_cfg), _P, _P, _P, _P, _P, _P]),
     "sd_denoise_workspace_size": (c_size_t, [POINTER(sd_unet_cfg)]),
@@ -225,6 +236,10 @@ def sd_unet_weight_layout(cfg):
     return _table(lib().sd_unet_weight_layout, ctypes.byref(cfg))
 
 
+def sd_vae_weight_layout(cfg):
+    return _table(lib().sd_vae_weight_layout, ctypes.byref(cfg))
+
+
 def _pack(fn, args, canonical_u16, packed_bytes):
     import numpy as np
     canon = np.ascontiguousarray(canonical_u16, dtype=np.uint16)
@@ -253,6 +268,10 @@ def sd_unet_pack_weights(cfg, canonical_u16, packed_bytes):
     return _pack(lib().sd_unet_pack_weights, (ctypes.byref(cfg),), canonical_u16, packed_bytes)
 
 
+def sd_vae_pack_weights(cfg, canonical_u16, packed_bytes):
+    return _pack(lib().sd_vae_pack_weights, (ctypes.byref(cfg),), canonical_u16, packed_bytes)
+
+
 # ---------------------------------------------------------------- workspace sizes
 
 def sd_time_workspace_size(cfg):
@@ -273,6 +292,10 @@ def sd_transformer_workspace_size(cfg):
 
 def sd_unet_workspace_size(cfg):
     return lib().sd_unet_workspace_size(ctypes.byref(cfg))
+
+
+def sd_vae_workspace_size(cfg):
+    return lib().sd_vae_workspace_size(ctypes.byref(cfg))
 
 
 # ---------------------------------------------------------------- forward calls
@@ -392,6 +415,12 @@ def sd_debug_inject_timeout(n_launches, spin_limit=1024):
     return _check(lib().sd_debug_inject_timeout(int(n_launches), int(spin_limit)), "sd_debug_inject_timeout")
 
 
+def sd_vae_decode(cfg, packed_w, latent, image, workspace, ws_bytes, stream=None, check=True):
+    s = lib().sd_vae_decode(ctypes.byref(cfg), _ptr(packed_w), _ptr(latent), _ptr(image), _ptr(workspace),
+                            int(ws_bytes), _stream(stream))
+    return _check(s, "sd_vae_decode") if check else s
+
+
 def sd_query_device_status(workspace, stream=None):
     return lib().sd_query_device_status(_ptr(workspace), _stream(stream))
 
@@ -452,6 +481,13 @@ def unet_cfg(in_channels=4, out_channels=4, height=96, width=96, block_channels=
     return sd_unet_cfg(in_channels, out_channels, height, width, len(block_channels), (c_int32 * 4)(*bc),
                        (c_int32 * 4)(*ad), layers_per_block, mid_depth, 64, ctx_len, ctx_dim, time_proj_dim,
                        temb_dim, groups, eps, add_text_dim, add_time_ids, add_time_dim)
+
+
+def vae_cfg(height, width, latent_channels=4, out_channels=3, block_channels=(128, 256, 512, 512),
+            layers_per_block=2, groups=32, eps=1e-5, scaling_factor=0.18215):
+    bc = list(block_channels) + [0] * (4 - len(block_channels))
+    return sd_vae_cfg(height, width, latent_channels, out_channels, len(block_channels), (c_int32 * 4)(*bc),
+                      layers_per_block, groups, eps, scaling_factor)
 
 
 def unet_cfg_from(ocfg, height, width):

@@ -55,7 +55,9 @@ sd_status device_info(DevInfo* out) {
 constexpr size_t kHeaderBytes = 256;   // word 0: device error flags
 constexpr int kMaxGnLaunches = 256;      // GroupNorm statistics slots per call
 constexpr int kMaxGroups = 64;
-constexpr size_t kGnAccBytes = (size_t)kMaxGnLaunches * 2 * kMaxGroups * sizeof(unsigned long long);
+// per GroupNorm launch: 2 * kMaxGroups sums, then the barrier counter of the single-pass kernel (padded)
+constexpr int kGnSlotWords = 2 * kMaxGroups + 2;
+constexpr size_t kGnAccBytes = (size_t)kMaxGnLaunches * kGnSlotWords * sizeof(unsigned long long);
 constexpr int kMaxStatBlocks = 512;  // GroupNorm partial-sum slots: 2 CTAs per SM, up to 256 SMs
 
 
@@ -75,7 +77,7 @@ struct Arena {
 struct Ctx {
   cudaStream_t st;
   int* err;
-  unsigned long long* gn_acc;  // [kMaxGnLaunches][2 * kMaxGroups], zeroed at the start of every call
+  unsigned long long* gn_acc;  // [kMaxGnLaunches][kGnSlotWords], zeroed at the start of every call
   int* gn_seq;                 // host: GroupNorm launches issued so far in this call
   float* skws;  // split-K FP32 partial products
   size_t skws_bytes;
@@ -140,9 +142,12 @@ int run_gemv(const Ctx& c, const sdk::GemvBatch& b) {
 sd_status run_gn(const Ctx& c, const bf16* x0, int C0, const bf16* x1, int C1, int HW, int G, float eps,
                  const bf16* gamma, const bf16* beta, int silu, bf16* y) {
   if (!c.gn_seq || *c.gn_seq >= kMaxGnLaunches) return SD_ERR_UNSUPPORTED;
-  unsigned long long* acc = c.gn_acc + (size_t)(*c.gn_seq)++ * 2 * kMaxGroups;
-  sdp::Scope sc("groupnorm", sdp::F_GN_APPLY, 0, 3.0 * HW * (C0 + C1) * 2, c.st, 2);
-  CK(sdk::launch_groupnorm(x0, C0, x1, C1, HW, G, eps, gamma, beta, silu, y, acc, c.sms, c.st));
+  unsigned long long* acc = c.gn_acc + (size_t)(*c.gn_seq)++ * kGnSlotWords;
+  unsigned int* counter = reinterpret_cast<unsigned int*>(acc + 2 * kMaxGroups);
+  const int nk = sdk::groupnorm_plan_launches(C0 + C1, HW, c.sms);
+  // algorithmic bytes: read once and write once (the two-kernel form reads twice)
+  sdp::Scope sc("groupnorm", sdp::F_GN_APPLY, 0, (nk == 1 ? 2.0 : 3.0) * HW * (C0 + C1) * 2, c.st, nk);
+  CK(sdk::launch_groupnorm(x0, C0, x1, C1, HW, G, eps, gamma, beta, silu, y, acc, counter, c.sms, c.st, c.err));
   return SD_OK;
 }
 
@@ -248,7 +253,7 @@ struct LnFold {
 
 sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, int N, const bf16* bias,
                      const bf16* residual, int ld_res, bf16* out, int ld_out, int mode = sdk::GEMM_PLAIN,
-                     double alg_k = 0, const LnFold* ln = nullptr) {
+                     double alg_k = 0, const LnFold* ln = nullptr, int f16_begin = 0) {
   GemmProblem p = base_problem(c);
   p.Ho = 1;
   p.Wo = M;
@@ -265,6 +270,7 @@ sd_status run_linear(const Ctx& c, const bf16* A, int M, int K, const bf16* B, i
   p.epi.out = out;
   p.epi.ld_out = ld_out;
   p.epi.mode = mode;
+  p.epi.f16_begin = f16_begin;
   if (ln) {
     p.epi.rowstat_out = ln->out;
     p.epi.rowstat_clear = ln->clear;
@@ -318,6 +324,15 @@ sd_status run_resblock(const Ctx& c, const ResW& w, const void* pw, int H, int W
   const int cout = w.c_out;
   const int rmod = t_rec.on ? t_rec.res_count++ : -1;
   sd_status r;
+  if (rmod >= 0) {
+    // the block input, so that h1 can be compared with a reference computed from the same input
+    bf16* d = rec_slot("x_h1", rmod, 0, HW, cx);
+    if (d && cudaMemcpyAsync(d, x, (size_t)HW * cx * 2, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+      return SD_ERR_LAUNCH;
+    bf16* e = cs > 0 ? rec_slot("x_skip", rmod, 0, HW, cs) : nullptr;
+    if (e && cudaMemcpyAsync(e, skip, (size_t)HW * cs * 2, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+      return SD_ERR_LAUNCH;
+  }
   // h1 = conv1(SiLU(GN1([x | skip]))) + b1 + tproj
   if ((r = run_gn(c, x, cx, skip, cs, HW, G, eps, W(pw, w.n1g), W(pw, w.n1b), 1, s.xn)) != SD_OK) return r;
   {
@@ -418,6 +433,14 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
     if (!d) return SD_OK;
     return run_linear(c, A, HW, K, W(pw, w_off), C, W(pw, b_off), nullptr, 0, d, C);
   };
+  // the residual stream entering a sublayer (the sublayer's input before its LayerNorm)
+  auto record_in = [&](const char* name) -> sd_status {
+    if (tmod < 0) return SD_OK;
+    bf16* d = rec_slot(name, tmod, bi, HW, C);
+    if (d && cudaMemcpyAsync(d, s.t, (size_t)HW * C * 2, cudaMemcpyDeviceToDevice, c.st) != cudaSuccess)
+      return SD_ERR_LAUNCH;
+    return SD_OK;
+  };
   // The three LayerNorms of each block are folded into the GEMMs they feed
   // (Q/K/V, the cross-attention query, FF1): every GEMM that writes the
   // residual stream t also leaves t's row sums in one of two buffers, and
@@ -458,10 +481,12 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
   }
   for (const TxBlockW& b : w.blocks) {
     // self-attention: t += Wo Attn(LN1(t)), LN1 folded into the Q/K/V GEMM
+    if ((r = record_in("x_attn1")) != SD_OK) return r;
     {
       const LnFold f = consumer(b.qkv_c1, b.qkv_c2);
+      // V (columns 2C..3C) is stored as FP16: the attention kernel multiplies it with FP16 probabilities
       if ((r = run_linear(c, s.t, HW, C, W(pw, b.qkv), 3 * C, nullptr, nullptr, 0, s.big, 3 * C, sdk::GEMM_PLAIN, 0,
-                          &f)) != SD_OK)
+                          &f, 2 * C)) != SD_OK)
         return r;
     }
     CK(run_attn(c, s.big, 3 * C, 0, s.big, 3 * C, C, 2 * C, s.ao, C, HW, HW, heads));
@@ -473,13 +498,15 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
         return r;
     }
     // cross-attention: t += Wo' Attn(LN2(t), ctx)
+    if ((r = record_in("x_attn2")) != SD_OK) return r;
     {
       const LnFold f = consumer(b.q2_c1, b.q2_c2);
       if ((r = run_linear(c, s.t, HW, C, W(pw, b.q2), C, nullptr, nullptr, 0, s.big, C, sdk::GEMM_PLAIN, 0, &f)) !=
           SD_OK)
         return r;
     }
-    if ((r = run_linear(c, ctx, ctx_len, w.ctx_dim, W(pw, b.kv2), 2 * C, nullptr, nullptr, 0, s.kv, 2 * C)) != SD_OK)
+    if ((r = run_linear(c, ctx, ctx_len, w.ctx_dim, W(pw, b.kv2), 2 * C, nullptr, nullptr, 0, s.kv, 2 * C,
+                        sdk::GEMM_PLAIN, 0, nullptr, C)) != SD_OK)  // V as FP16
       return r;
     CK(run_attn(c, s.big, C, 0, s.kv, 2 * C, 0, C, s.ao, C, HW, ctx_len, heads));
     if ((r = record("attn2", s.ao, C, b.o2w, b.o2b)) != SD_OK) return r;
@@ -490,6 +517,7 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
         return r;
     }
     // GEGLU feed-forward: t += W2 (a * GELU(g)) + b2, LN3 folded into FF1 (its bias is in c2)
+    if ((r = record_in("x_ff")) != SD_OK) return r;
     {
       const LnFold f = consumer(b.f1_c1, b.f1_c2);
       if ((r = run_linear(c, s.t, HW, C, W(pw, b.f1w), 8 * C, nullptr, nullptr, 0, s.big, 4 * C, sdk::GEMM_GEGLU, 0,
@@ -592,6 +620,63 @@ sd_status run_time(const Ctx& c, const TimeW& w, const void* pw, int proj, int t
   return SD_OK;
 }
 
+// Single-head self-attention of the VAE MidBlock over the H*W tokens:
+// y = x + (softmax(Q K^T / sqrt(C)) V) W_o^T + b_o with Q, K, V from GN(x). The
+// head is C = 512 wide, so the scores are formed explicitly: an FP32 [HW, HW]
+// score GEMM (Q against the K columns of the same matrix), a row softmax to
+// BF16 probabilities, V transposed once, and the probability GEMM.
+struct VaeAttnScratch {
+  bf16 *nrm, *qkv, *vt, *o, *p;
+  float* s;
+};
+VaeAttnScratch plan_vae_attn_scratch(Arena& ar, int64_t HW, int C) {
+  VaeAttnScratch v;
+  v.nrm = ar.bf((size_t)HW * C);
+  v.qkv = ar.bf((size_t)HW * 3 * C);
+  v.vt = ar.bf((size_t)HW * C);
+  v.o = ar.bf((size_t)HW * C);
+  v.p = ar.bf((size_t)HW * HW);
+  v.s = ar.f32((size_t)HW * HW);
+  return v;
+}
+
+sd_status run_vae_attention(const Ctx& c, const VaeAttnW& w, const void* pw, int H, int Wd, int G, float eps,
+                            const bf16* x, bf16* y, const VaeAttnScratch& s) {
+  const int HW = H * Wd;
+  const int C = w.C;
+  sd_status r;
+  if ((r = run_gn(c, x, C, nullptr, 0, HW, G, eps, W(pw, w.ng), W(pw, w.nb), 0, s.nrm)) != SD_OK) return r;
+  if ((r = run_linear(c, s.nrm, HW, C, W(pw, w.qkv), 3 * C, W(pw, w.qkv_b), nullptr, 0, s.qkv, 3 * C)) != SD_OK)
+    return r;
+  {
+    // S = Q K^T: A = the Q columns of qkv, B = the K columns of the same matrix (rows = keys)
+    GemmProblem p = base_problem(c);
+    p.Ho = 1;
+    p.Wo = HW;
+    p.N = HW;
+    p.na = 1;
+    p.a[0] = {s.qkv, 3 * C, HW, 1, 1};
+    p.nb = 1;
+    p.b[0] = {s.qkv, 3 * C, HW};
+    p.nseg = 1;
+    p.seg[0] = {0, 0, 0, 0, 0, 0, C, C / 64};
+    p.epi.out = reinterpret_cast<bf16*>(s.s);
+    p.epi.ld_out = HW;
+    p.epi.mode = sdk::GEMM_F32;
+    CK(launch_gemm(c, p));
+  }
+  {
+    sdp::Scope sc("softmax_rows", sdp::F_OTHER, 0, (double)HW * HW * 6.0, c.st);
+    CK(sdk::launch_softmax_rows(s.s, HW, HW, HW, 1.0f / sqrtf((float)C), s.p, HW, c.st));
+  }
+  {
+    sdp::Scope sc("transpose", sdp::F_OTHER, 0, 4.0 * HW * C, c.st);
+    CK(sdk::launch_transpose(s.qkv, 3 * C, 2 * C, HW, C, s.vt, HW, c.st));
+  }
+  if ((r = run_linear(c, s.p, HW, HW, s.vt, C, nullptr, nullptr, 0, s.o, C)) != SD_OK) return r;
+  return run_linear(c, s.o, HW, C, W(pw, w.ow), C, W(pw, w.ob), x, C, y, C);
+}
+
 // ------------------------------------------------------------------ validation helpers
 bool ch_ok(int c) { return c > 0 && c % 64 == 0; }
 bool groups_ok(int C, int G) { return G > 0 && G <= kMaxGroups && C % G == 0 && C / G >= 8; }
@@ -668,6 +753,28 @@ sd_status check_unet(const sd_unet_cfg* cfg) {
     if (!ch_ok(cfg->block_channels[l]) || cfg->block_channels[l] > 2048) return SD_ERR_UNSUPPORTED;
     if (!groups_ok(cfg->block_channels[l], cfg->groups) || cfg->attn_depth[l] < 0) return SD_ERR_UNSUPPORTED;
   }
+  return SD_OK;
+}
+
+sd_status check_vae(const sd_vae_cfg* cfg) {
+  if (!cfg) return SD_ERR_NULL_ARG;
+  const int L = cfg->n_levels;
+  if (L < 1 || L > 4 || cfg->layers_per_block < 0 || cfg->layers_per_block > 7) return SD_ERR_UNSUPPORTED;
+  if (cfg->latent_channels < 1 || cfg->latent_channels > 16 || cfg->out_channels < 1 || cfg->out_channels > 16)
+    return SD_ERR_UNSUPPORTED;
+  if (cfg->height <= 0 || cfg->width <= 0) return SD_ERR_BAD_SHAPE;
+  if ((cfg->height * cfg->width) % 64) return SD_ERR_UNSUPPORTED;  // the attention's token count is a K dimension
+  if (!(cfg->scaling_factor > 0.f)) return SD_ERR_BAD_SHAPE;
+  for (int l = 0; l < L; ++l) {
+    const int C = cfg->block_channels[l];
+    if (!ch_ok(C) || C > 2048) return SD_ERR_UNSUPPORTED;
+    // GroupNorm: at least 8 channels per group, or exactly 4 (an 8-channel vector then covers two whole groups)
+    const int G = cfg->groups;
+    if (G <= 0 || G > kMaxGroups || C % G || (C / G < 8 && C / G != 4)) return SD_ERR_UNSUPPORTED;
+  }
+  // the full score matrix of the MidBlock attention lives in the workspace (FP32 + BF16)
+  const int64_t hw = (int64_t)cfg->height * cfg->width;
+  if (hw > 16384 * 4) return SD_ERR_UNSUPPORTED;
   return SD_OK;
 }
 
@@ -826,6 +933,53 @@ size_t plan_unet(Arena& ar, const sd_unet_cfg* cfg, cudaStream_t st, int sms, UN
   uint8_t* sh = static_cast<uint8_t*>(ar.take(shared + 4096));
   p->conv_scratch = reinterpret_cast<bf16*>(sh);
   (void)sh;
+  return ar.off;
+}
+
+struct VaePlan {
+  Ctx c;
+  bf16 *pp[2];
+  bf16* shared;  // resblock / attention / resampling / conv_in scratch, used one at a time
+  size_t shared_bytes;
+};
+
+size_t plan_vae(Arena& ar, const sd_vae_cfg* cfg, cudaStream_t st, int sms, VaePlan* p) {
+  const int L = cfg->n_levels;
+  std::vector<int> ch;
+  for (int l = L - 1; l >= 0; --l) ch.push_back(cfg->block_channels[l]);
+  p->c = make_ctx(ar, st, sms);
+  auto rnd = [](size_t b) { return (b + 255) / 256 * 256; };
+  size_t H = cfg->height, Wd = cfg->width;
+  size_t max_act = H * Wd * ch[0];
+  size_t need = rnd(H * Wd * cfg->latent_channels * 2) + rnd(H * Wd * conv_in_kp(cfg->latent_channels) * 2);
+  {
+    Arena a{nullptr, 0};
+    plan_vae_attn_scratch(a, (int64_t)(H * Wd), ch[0]);
+    need = std::max(need, a.off + 1024);
+  }
+  int c_prev = ch[0];
+  auto res_need = [&](size_t hw, int ci, int co) {
+    need = std::max(need, rnd(hw * ci * 2) + 2 * rnd(hw * co * 2) + 1024);
+    max_act = std::max(max_act, hw * (size_t)co);
+  };
+  res_need(H * Wd, c_prev, c_prev);
+  for (int i = 0; i < L; ++i) {
+    for (int j = 0; j <= cfg->layers_per_block; ++j) {
+      res_need(H * Wd, c_prev, ch[i]);
+      c_prev = ch[i];
+    }
+    if (i < L - 1) {
+      need = std::max(need, rnd(4 * H * Wd * ch[i] * 2) + 1024);  // materialised nearest-2x input
+      H *= 2;
+      Wd *= 2;
+      max_act = std::max(max_act, H * Wd * (size_t)ch[i]);
+    }
+  }
+  need = std::max(need, rnd(H * Wd * ch[L - 1] * 2) + 1024);  // output head GroupNorm
+  p->pp[0] = ar.bf(max_act);
+  p->pp[1] = ar.bf(max_act);
+  p->shared = static_cast<bf16*>(ar.take(need));
+  p->shared_bytes = need;
   return ar.off;
 }
 
@@ -1316,6 +1470,102 @@ sd_status sd_unet_step_cond(const sd_unet_cfg* cfg, const void* pw, const void* 
   }
   return run_output(c, u.out, pw, H, Wd, hc, cfg->out_channels, G, eps, h, static_cast<bf16*>(eps_out),
                     reinterpret_cast<bf16*>(shared));
+}
+
+sd_status sd_vae_weight_layout(const sd_vae_cfg* cfg, sd_tensor_desc* out, int32_t capacity, int32_t* n, int64_t* ce,
+                               int64_t* pb) {
+  sd_status s = check_vae(cfg);
+  if (s != SD_OK) return s;
+  Table t;
+  add_vae(t, *cfg);
+  return export_table(t, out, capacity, n, ce, pb);
+}
+
+sd_status sd_vae_pack_weights(const sd_vae_cfg* cfg, const uint16_t* canon, void* packed) {
+  sd_status s = check_vae(cfg);
+  if (s != SD_OK) return s;
+  if (!canon || !packed) return SD_ERR_NULL_ARG;
+  Table t;
+  add_vae(t, *cfg);
+  pack(t, canon, static_cast<uint8_t*>(packed));
+  return SD_OK;
+}
+
+size_t sd_vae_workspace_size(const sd_vae_cfg* cfg) {
+  if (check_vae(cfg) != SD_OK) return 0;
+  Arena a{nullptr, 0};
+  VaePlan p;
+  return plan_vae(a, cfg, nullptr, kMaxStatBlocks, &p);
+}
+
+sd_status sd_vae_decode(const sd_vae_cfg* cfg, const void* pw, const void* latent, void* image, void* ws,
+                        size_t ws_bytes, sd_stream_t stream) {
+  sd_status s = check_vae(cfg);
+  if (s != SD_OK) return s;
+  if (!pw || !latent || !image) return SD_ERR_NULL_ARG;
+  if (!aligned16(pw) || !aligned16(latent) || !aligned16(image)) return SD_ERR_MISALIGNED;
+  if ((s = check_ws(sd_vae_workspace_size(cfg), ws, ws_bytes)) != SD_OK) return s;
+  DevInfo d;
+  if ((s = device_info(&d)) != SD_OK) return s;
+  Arena a{static_cast<uint8_t*>(ws), 0};
+  VaePlan p;
+  plan_vae(a, cfg, (cudaStream_t)stream, d.sms, &p);
+  const Ctx& c = p.c;
+  if ((s = clear_header(c)) != SD_OK) return s;
+  int gn_seq = 0;
+  p.c.gn_seq = &gn_seq;
+  Table tab;
+  const VaeW v = add_vae(tab, *cfg);
+  const int G = cfg->groups, L = cfg->n_levels;
+  const float eps = cfg->eps;
+  int H = cfg->height, Wd = cfg->width;
+  uint8_t* sh = reinterpret_cast<uint8_t*>(p.shared);
+  // latent / scaling factor -> 1x1 post-quantisation conv -> conv_in
+  {
+    const int lc = cfg->latent_channels;
+    bf16* lat = reinterpret_cast<bf16*>(sh);
+    bf16* col = reinterpret_cast<bf16*>(sh + ((size_t)H * Wd * lc * 2 + 255) / 256 * 256);
+    {
+      sdp::Scope sc("vae_latent_in", sdp::F_OTHER, 0, 4.0 * H * Wd * lc, c.st);
+      CK(sdk::launch_vae_latent_in(static_cast<const bf16*>(latent), W(pw, v.post_quant.w), W(pw, v.post_quant.b), lc,
+                                   (int64_t)H * Wd, 1.0f / cfg->scaling_factor, lat, c.st));
+    }
+    if ((s = run_conv_in(c, v.conv_in, pw, v.conv_in_kp, H, Wd, lat, lc, nullptr, 0, nullptr, 0,
+                         v.up[0].C, p.pp[0], col)) != SD_OK)
+      return s;
+  }
+  int cur = 0;
+  auto res = [&](const ResW& w, int cx) -> sd_status {
+    ResScratch rs = carve_res(sh, H * Wd, cx, w.c_out);
+    sd_status r = run_resblock(c, w, pw, H, Wd, p.pp[cur], cx, nullptr, 0, nullptr, G, eps, p.pp[cur ^ 1], rs);
+    cur ^= 1;
+    return r;
+  };
+  int C = v.up[0].C;
+  if ((s = res(v.mid_res0, C)) != SD_OK) return s;
+  {
+    Arena aa{sh, 0};
+    const VaeAttnScratch as = plan_vae_attn_scratch(aa, (int64_t)H * Wd, C);
+    if ((s = run_vae_attention(c, v.mid_attn, pw, H, Wd, G, eps, p.pp[cur], p.pp[cur ^ 1], as)) != SD_OK) return s;
+    cur ^= 1;
+  }
+  if ((s = res(v.mid_res1, C)) != SD_OK) return s;
+  for (int i = 0; i < L; ++i) {
+    for (const ResW& w : v.up[i].res) {
+      if ((s = res(w, C)) != SD_OK) return s;
+      C = w.c_out;
+    }
+    if (v.up[i].has_up) {
+      if ((s = run_upsample(c, v.up[i].up, pw, H, Wd, C, p.pp[cur], p.pp[cur ^ 1], reinterpret_cast<bf16*>(sh))) !=
+          SD_OK)
+        return s;
+      cur ^= 1;
+      H *= 2;
+      Wd *= 2;
+    }
+  }
+  return run_output(c, v.out, pw, H, Wd, C, cfg->out_channels, G, eps, p.pp[cur], static_cast<bf16*>(image),
+                    reinterpret_cast<bf16*>(sh));
 }
 
 sd_status sd_record_begin(void* dev_buf, size_t bytes) {

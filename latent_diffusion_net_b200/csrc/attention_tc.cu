@@ -17,17 +17,23 @@
 // 192 threads per CTA:
 //   warps 0-3  softmax: thread i owns query row i (TMEM lane i). Per 128-key
 //              tile it reads its S row from TMEM, keeps a running maximum in the
-//              log2 domain, writes P = exp2(s*log2e/8 - m) as BF16 into shared
-//              memory (the A operand of the PV product, 128-byte swizzled), and
-//              accumulates the row sum in a register. The output O lives in TMEM
-//              and is rescaled only when the running maximum grew by more than
-//              2^8 since the last rescale (P values stay <= 256, exact in FP32).
+//              log2 domain, and forms P = exp2(s*log2e/8 - m) two at a time: the
+//              pair of FP32 exponents is rounded to FP16 and one packed
+//              ex2.approx.f16x2 gives both probabilities, already in the FP16
+//              form the PV product takes (so one exponential-unit issue serves
+//              two keys and no conversion follows). P goes to shared memory (the
+//              A operand of the PV product, 128-byte swizzled); the row sum is
+//              kept in four packed FP16 partial sums per tile, added into FP32
+//              once per tile. The output O lives in TMEM and is rescaled only
+//              when the running maximum grew by more than 2^8 since the last
+//              rescale (P values stay <= 256).
 //   warp 4     TMA producer: Q once per item, K tiles (double-buffered) and V
 //              tiles (single buffer, reloaded once the previous PV product is
-//              done), zero-filled past the last key.
-//   warp 5     MMA issuer (one thread): S = Q K^T (M=128, N=128, K=64) and
-//              O += P V (M=128, N=64, K=128, V read MN-major), both
-//              tcgen05.mma kind::f16, BF16 in, FP32 accumulate in TMEM.
+//              done), zero-filled past the last key. V arrives as FP16 (the
+//              projection GEMM stores those columns in FP16).
+//   warp 5     MMA issuer (one thread): S = Q K^T (M=128, N=128, K=64, BF16) and
+//              O += P V (M=128, N=64, K=128, FP16, V read MN-major), both
+//              tcgen05.mma kind::f16 with FP32 accumulation in TMEM.
 // TMEM: S in columns [0, 128), O in [128, 192) of a 256-column allocation, so
 // two CTAs fit on one SM and overlap each other's softmax and MMA phases.
 #include "common.cuh"
@@ -48,10 +54,10 @@ constexpr int kTileBytes = 128 * 64 * 2;  // one [128 x 64] BF16 tile = 16 KB
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kOCol = 128;
 
-// Instruction descriptor: BF16 x BF16 -> FP32, M = 128, A K-major, B K-major
-// (S = Q K^T) or B MN-major (O += P V).
-__host__ __device__ constexpr uint32_t idesc_attn(int N, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+// Instruction descriptor, FP32 accumulator, M = 128, A K-major: BF16 x BF16 with
+// B K-major (S = Q K^T), or FP16 x FP16 with B MN-major (O += P V).
+__host__ __device__ constexpr uint32_t idesc_attn(int N, bool pv) {
+  return (1u << 4) | (pv ? 0u : (1u << 7) | (1u << 10)) | ((pv ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(128 >> 4) << 24);
 }
 
@@ -68,13 +74,29 @@ __device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t smem_addr) {
   return d;
 }
 
-// BF16 pair by integer rounding (half away from zero in magnitude) on the ALU
-// pipe, leaving the conversion unit free for the exponentials; inputs are
-// finite and non-negative here.
-__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo) + 0x8000u;
-  const uint32_t b = __float_as_uint(hi) + 0x8000u;
-  return __byte_perm(a, b, 0x7632);
+// Two FP32 values rounded to one packed FP16 pair (lo in the low half).
+__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// 2^x for both halves of a packed FP16 pair (one exponential-unit instruction).
+__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t x) {
+  uint32_t y;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t add_f16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ float f16x2_sum(uint32_t h) {
+  const __half2 v = *reinterpret_cast<const __half2*>(&h);
+  return __low2float(v) + __high2float(v);
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -360,17 +382,24 @@ __global__ void __launch_bounds__(192, 2)
           rescale = true;
         }
       }
-      // P = exp2(s*scale*log2e - m_used) as packed BF16 pairs in registers (masked keys give
-      // exp2(-inf) = 0) while the previous PV product may still be running; row sum in two chains
+      // P = exp2(s*scale*log2e - m_used) as packed FP16 pairs in registers (masked keys give
+      // exp2(-inf) = 0) while the previous PV product may still be running; the row sum in
+      // four packed FP16 partial sums of 16 pairs each (every P <= 256, so no partial sum
+      // exceeds 4096)
       uint32_t pk[64];
-      float la = 0.f, lb = 0.f;
+      uint32_t hs0 = 0u, hs1 = 0u, hs2 = 0u, hs3 = 0u;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2(fmaf(__uint_as_float(sv[2 * i]), sl2, -m_used));
-        const float p1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -m_used));
-        la += p0;
-        lb += p1;
-        pk[i] = pack_bf16x2_alu(p0, p1);
+      for (int i = 0; i < 64; i += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float x0 = fmaf(__uint_as_float(sv[2 * (i + u)]), sl2, -m_used);
+          const float x1 = fmaf(__uint_as_float(sv[2 * (i + u) + 1]), sl2, -m_used);
+          pk[i + u] = ex2_f16x2(cvt_f16x2(x0, x1));
+        }
+        hs0 = add_f16x2(hs0, pk[i]);
+        hs1 = add_f16x2(hs1, pk[i + 1]);
+        hs2 = add_f16x2(hs2, pk[i + 2]);
+        hs3 = add_f16x2(hs3, pk[i + 3]);
       }
       // the previous PV product must be done before P is overwritten or O rescaled
       if (t > 0 && !mbar_wait(pv_done, (t - 1) & 1, abort_flag, args.err)) break;
@@ -400,7 +429,7 @@ __global__ void __launch_bounds__(192, 2)
                        : "memory");
         }
       }
-      l += la + lb;
+      l += (f16x2_sum(hs0) + f16x2_sum(hs1)) + (f16x2_sum(hs2) + f16x2_sum(hs3));
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);

@@ -327,8 +327,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const __nv_bfloat16* const bias2 = args.epi.bias2;
     const float* const colvec = args.epi.colvec;
     const __nv_bfloat16* const residual = args.epi.residual;
-    const int ld_res = args.epi.ld_res, ld_out = args.epi.ld_out;
+    const int ld_res = args.epi.ld_res, ld_out = args.epi.ld_out, f16_begin = args.epi.f16_begin;
     const bool geglu = args.epi.mode == GEMM_GEGLU;
+    const bool f32_out = args.epi.mode == GEMM_F32;
     __nv_bfloat16* const out = args.epi.out;
     const bool has_cols = partial == nullptr && (bias || bias2 || colvec);
     unsigned long long* const rowstat_out = args.epi.rowstat_out;
@@ -430,8 +431,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
         }
         const bool full = (nb + 32 <= N);
-        if (partial) {
-          float* dst = partial + ((size_t)z * Ho * Wo + grow) * N + nb;
+        if (partial || f32_out) {
+          float* dst = partial ? partial + ((size_t)z * Ho * Wo + grow) * N + nb
+                               : reinterpret_cast<float*>(out) + grow * ld_out + nb;
           if (full) {
             float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
@@ -491,7 +493,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
         __nv_bfloat16* dst = out + grow * ld_out + nb;
-        if (full) {
+        if (full && f16_begin > 0 && nb >= f16_begin) {
+          // FP16 columns (the attention values V; no row statistics are taken over them)
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            d4[w] = make_uint4(pack_f16x2(v[8 * w + 0], v[8 * w + 1]), pack_f16x2(v[8 * w + 2], v[8 * w + 3]),
+                               pack_f16x2(v[8 * w + 4], v[8 * w + 5]), pack_f16x2(v[8 * w + 6], v[8 * w + 7]));
+          }
+        } else if (full) {
           uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
@@ -580,6 +590,11 @@ __device__ __forceinline__ void splitk_reduce_vec(const float* __restrict__ part
     const uint4 r = *reinterpret_cast<const uint4*>(epi.residual + (size_t)row * epi.ld_res + c);
     v[0] += bf16lo(r.x); v[1] += bf16hi(r.x); v[2] += bf16lo(r.y); v[3] += bf16hi(r.y);
     v[4] += bf16lo(r.z); v[5] += bf16hi(r.z); v[6] += bf16lo(r.w); v[7] += bf16hi(r.w);
+  }
+  if (epi.f16_begin > 0 && c >= epi.f16_begin) {
+    *reinterpret_cast<uint4*>(epi.out + (size_t)row * epi.ld_out + c) =
+        make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
+    return;
   }
   const uint4 o = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                              pack_bf16x2(v[6], v[7]));
@@ -898,7 +913,8 @@ static bool plan_gemm(const GemmProblem& p, GemmPlan* g) {
       } else if (sp > 1 && (g->total_kb / sp < 2 || (sp > 8 && sp % 2))) {
         continue;
       }
-      if (sp > 1 && (!p.splitk_ws || per_split * sp > p.splitk_ws_bytes || p.N % 8)) continue;
+      if (sp > 1 && (!p.splitk_ws || per_split * sp > p.splitk_ws_bytes || p.N % 8 || p.epi.mode == GEMM_F32))
+        continue;
       const double c = plan_cost(*g, bn, sp, pairs, p.N, M, max_clusters);
       if (best < 0 || c < best) {
         best = c;

@@ -15,7 +15,9 @@ constexpr int kGemmMaxSeg = 12;
 constexpr int kGemmMaxA = 4;
 constexpr int kGemmMaxB = 2;
 
-enum GemmMode : int32_t { GEMM_PLAIN = 0, GEMM_GEGLU = 1 };
+// GEMM_F32: the output (after the biases) is stored as FP32 to (float*)out with
+// row stride ld_out elements; no residual, no split reduction.
+enum GemmMode : int32_t { GEMM_PLAIN = 0, GEMM_GEGLU = 1, GEMM_F32 = 2 };
 
 // One activation source: a BF16 NHWC tensor seen as [Z][H][W][C].
 struct GemmASrc {
@@ -47,6 +49,7 @@ struct GemmEpi {
   __nv_bfloat16* out;             // [M][ld_out]
   int32_t ld_out;
   int32_t mode;                   // GemmMode
+  int32_t f16_begin;              // > 0: output columns >= f16_begin are stored as FP16 (a multiple of 32)
   // Row statistics for a LayerNorm folded into the next GEMM. rowstat_out: each
   // output row's sum and sum of squares of the stored BF16 values are added into
   // rowstat_out[2*row .. 2*row+1] as 64-bit fixed point (scales 2^24 and 2^18);

@@ -8,11 +8,16 @@
 namespace sdk {
 
 // GroupNorm (+SiLU) of the channel concatenation [x0 | x1] (x1 may be null with
-// C1 = 0) into y: a statistics kernel and an apply kernel. `acc` holds 2*G
-// zero-initialised 64-bit words used by this call only.
+// C1 = 0) into y. `acc` holds 2*G and `counter` one zero-initialised word used
+// by this call only. When each CTA's share of the pixels fits in shared memory
+// one kernel does both passes (statistics, grid barrier, normalisation; a
+// barrier that times out raises ERR_MBAR_TIMEOUT in *err); otherwise a
+// statistics kernel and an apply kernel run (counter / err may then be null).
 int launch_groupnorm(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G, float eps,
                      const __nv_bfloat16* gamma, const __nv_bfloat16* beta, int silu, __nv_bfloat16* y,
-                     unsigned long long* acc, int num_sms, cudaStream_t st);
+                     unsigned long long* acc, unsigned int* counter, int num_sms, cudaStream_t st, int* err);
+// Kernels launch_groupnorm enqueues for these sizes (1 or 2).
+int groupnorm_plan_launches(int C, int HW, int num_sms);
 // Time embedding: phi(t) sinusoid [proj_dim] into out (FP32).
 int launch_sinusoid(float t, int proj_dim, float* out, cudaStream_t st);
 
@@ -41,6 +46,17 @@ struct AddIds {
 };
 int launch_add_embed_input(const __nv_bfloat16* text, int text_dim, const AddIds& ids, int n_ids, int dim,
                            float* out, cudaStream_t st);
+
+// VAE decoder input: y = 1x1 conv (W [lc][lc], b [lc]) of z * inv_scale, NHWC [hw][lc].
+int launch_vae_latent_in(const __nv_bfloat16* z, const __nv_bfloat16* w, const __nv_bfloat16* b, int lc, int64_t hw,
+                         float inv_scale, __nv_bfloat16* y, cudaStream_t st);
+// Row softmax: P[r][:] = softmax(scale * S[r][:]) as BF16 for rows x n FP32 scores
+// (n a multiple of 8, at most 51200). Returns -1 for unsupported sizes.
+int launch_softmax_rows(const float* S, int64_t ld_s, int rows, int n, float scale, __nv_bfloat16* P, int64_t ld_p,
+                        cudaStream_t st);
+// dst[c][r] = src[r][c0 + c] (BF16), rows x cols.
+int launch_transpose(const __nv_bfloat16* src, int64_t ld_src, int c0, int rows, int cols, __nv_bfloat16* dst,
+                     int64_t ld_dst, cudaStream_t st);
 
 // Nearest 2x upsample of NHWC [H, W, C] into [2H, 2W, C].
 int launch_upsample2x(const __nv_bfloat16* x, int H, int W, int C, __nv_bfloat16* y, cudaStream_t st);

@@ -100,6 +100,117 @@ int launch_add_embed_input(const __nv_bfloat16* text, int text_dim, const AddIds
                          n_ids, dim, out);
 }
 
+// VAE decoder input: y[p][o] = b[o] + sum_c W[o][c] * (z[p][c] * inv_scale), the
+// latent divided by the scaling factor, then the 1x1 post-quantisation conv.
+__global__ void vae_latent_in_kernel(const __nv_bfloat16* __restrict__ z, const __nv_bfloat16* __restrict__ w,
+                                     const __nv_bfloat16* __restrict__ b, int lc, int64_t hw, float inv_scale,
+                                     __nv_bfloat16* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t total = hw * lc;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t p = i / lc;
+    const int o = (int)(i % lc);
+    float acc = __bfloat162float(b[o]);
+    for (int c = 0; c < lc; ++c)
+      acc = fmaf(__bfloat162float(w[o * lc + c]), __bfloat162float(z[p * lc + c]) * inv_scale, acc);
+    y[i] = __float2bfloat16_rn(acc);
+  }
+}
+
+int launch_vae_latent_in(const __nv_bfloat16* z, const __nv_bfloat16* w, const __nv_bfloat16* b, int lc, int64_t hw,
+                         float inv_scale, __nv_bfloat16* y, cudaStream_t st) {
+  const int64_t total = hw * lc;
+  int blocks = (int)((total + 255) / 256);
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  return (int)launch_pdl(vae_latent_in_kernel, dim3(blocks), dim3(256), 0, st, z, w, b, lc, hw, inv_scale, y);
+}
+
+// Row softmax of FP32 scores: P[r][j] = exp(scale*(S[r][j] - max_j S[r][j])) / sum, as BF16.
+// One CTA per row; the row is read once into shared memory.
+__global__ void __launch_bounds__(256) softmax_rows_kernel(const float* __restrict__ S, int64_t ld_s, int n,
+                                                           float scale_log2, __nv_bfloat16* __restrict__ P,
+                                                           int64_t ld_p) {
+  extern __shared__ float row[];
+  __shared__ float red[8];
+  pdl_wait();
+  pdl_trigger();
+  const float* src = S + (int64_t)blockIdx.x * ld_s;
+  float mx = -INFINITY;
+  for (int j = threadIdx.x * 4; j < n; j += blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(src + j);
+    *reinterpret_cast<float4*>(row + j) = v;
+    mx = fmaxf(fmaxf(mx, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
+  }
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[wid] = mx;
+  __syncthreads();
+  mx = red[0];
+  for (int k = 1; k < (int)(blockDim.x >> 5); ++k) mx = fmaxf(mx, red[k]);
+  __syncthreads();
+  const float m = mx * scale_log2;
+  float sum = 0.f;
+  for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    const float e = exp2f(fmaf(row[j], scale_log2, -m));
+    row[j] = e;
+    sum += e;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) red[wid] = sum;
+  __syncthreads();
+  float tot = 0.f;
+  for (int k = 0; k < (int)(blockDim.x >> 5); ++k) tot += red[k];
+  const float inv = 1.f / tot;
+  __nv_bfloat16* dst = P + (int64_t)blockIdx.x * ld_p;
+  for (int j = threadIdx.x * 8; j < n; j += blockDim.x * 8) {
+    *reinterpret_cast<uint4*>(dst + j) =
+        make_uint4(pack_bf16x2(row[j] * inv, row[j + 1] * inv), pack_bf16x2(row[j + 2] * inv, row[j + 3] * inv),
+                   pack_bf16x2(row[j + 4] * inv, row[j + 5] * inv), pack_bf16x2(row[j + 6] * inv, row[j + 7] * inv));
+  }
+}
+
+int launch_softmax_rows(const float* S, int64_t ld_s, int rows, int n, float scale, __nv_bfloat16* P, int64_t ld_p,
+                        cudaStream_t st) {
+  if (n % 8 || ld_s % 4 || ld_p % 8) return -1;
+  const size_t smem = (size_t)n * sizeof(float);
+  if (smem > 200 * 1024) return -1;
+  static bool attr = false;  // benign race: identical value for every caller
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(softmax_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e != cudaSuccess) return (int)e;
+    attr = true;
+  }
+  return (int)launch_pdl(softmax_rows_kernel, dim3(rows), dim3(256), smem, st, S, ld_s, n,
+                         scale * 1.4426950408889634f, P, ld_p);
+}
+
+// dst[c][r] = src[r][c0 + c] for r < rows, c < cols (32 x 32 tiles through shared memory).
+__global__ void transpose_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld_src, int c0, int rows, int cols,
+                                 __nv_bfloat16* __restrict__ dst, int64_t ld_dst) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  pdl_wait();
+  pdl_trigger();
+  const int r0 = blockIdx.y * 32, cb = blockIdx.x * 32;
+  for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+    const int r = r0 + k, c = cb + threadIdx.x;
+    if (r < rows && c < cols) tile[k][threadIdx.x] = src[(int64_t)r * ld_src + c0 + c];
+  }
+  __syncthreads();
+  for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+    const int c = cb + k, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) dst[(int64_t)c * ld_dst + r] = tile[threadIdx.x][k];
+  }
+}
+
+int launch_transpose(const __nv_bfloat16* src, int64_t ld_src, int c0, int rows, int cols, __nv_bfloat16* dst,
+                     int64_t ld_dst, cudaStream_t st) {
+  return (int)launch_pdl(transpose_kernel, dim3((cols + 31) / 32, (rows + 31) / 32), dim3(32, 8), 0, st, src, ld_src,
+                         c0, rows, cols, dst, ld_dst);
+}
+
 // Nearest 2x (UpSample bullet): y[i][j] = x[i/2][j/2], one 16-byte vector per thread.
 __global__ void upsample2x_kernel(const uint4* __restrict__ x, int H, int W, int V, uint4* __restrict__ y) {
   pdl_wait();

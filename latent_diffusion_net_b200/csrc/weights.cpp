@@ -206,6 +206,71 @@ UNetW add_unet(Table& tab, const sd_unet_cfg& cfg) {
   return u;
 }
 
+static ResW add_vae_resblock(Table& tab, const std::string& p, int ci, int co) {
+  ResW w;
+  w.c_in = ci;
+  w.c_out = co;
+  w.n1g = tab.add(p + ".norm1.gamma", {ci}, SD_KIND_NORM_GAMMA, 0);
+  w.n1b = tab.add(p + ".norm1.beta", {ci}, SD_KIND_NORM_BETA, 0);
+  w.c1w = tab.add(p + ".conv1.weight", {co, ci, 3, 3}, SD_KIND_WEIGHT, ci * 9, PACK_CONV_KRSC);
+  w.c1b = tab.add(p + ".conv1.bias", {co}, SD_KIND_BIAS, ci * 9);
+  w.tw = w.tb = -1;
+  w.n2g = tab.add(p + ".norm2.gamma", {co}, SD_KIND_NORM_GAMMA, 0);
+  w.n2b = tab.add(p + ".norm2.beta", {co}, SD_KIND_NORM_BETA, 0);
+  w.c2w = tab.add(p + ".conv2.weight", {co, co, 3, 3}, SD_KIND_WEIGHT, co * 9, PACK_CONV_KRSC);
+  w.c2b = tab.add(p + ".conv2.bias", {co}, SD_KIND_BIAS, co * 9);
+  w.sw = w.sb = -1;
+  if (ci != co) {
+    w.sw = tab.add(p + ".skip.weight", {co, ci, 1, 1}, SD_KIND_WEIGHT, ci);
+    w.sb = tab.add(p + ".skip.bias", {co}, SD_KIND_BIAS, ci);
+  }
+  return w;
+}
+
+VaeW add_vae(Table& tab, const sd_vae_cfg& cfg) {
+  VaeW v;
+  const int L = cfg.n_levels;
+  const int lc = cfg.latent_channels;
+  std::vector<int> ch;
+  for (int l = L - 1; l >= 0; --l) ch.push_back(cfg.block_channels[l]);
+  v.post_quant.w = tab.add("post_quant_conv.weight", {lc, lc, 1, 1}, SD_KIND_WEIGHT, lc);
+  v.post_quant.b = tab.add("post_quant_conv.bias", {lc}, SD_KIND_BIAS, lc);
+  v.conv_in_kp = conv_in_kp(lc);
+  v.conv_in = add_conv_in(tab, "conv_in", lc, ch[0], v.conv_in_kp);
+  v.mid_res0 = add_vae_resblock(tab, "mid.res.0", ch[0], ch[0]);
+  {
+    const int C = ch[0];
+    VaeAttnW& a = v.mid_attn;
+    a.C = C;
+    a.ng = tab.add("mid.attn.norm.gamma", {C}, SD_KIND_NORM_GAMMA, 0);
+    a.nb = tab.add("mid.attn.norm.beta", {C}, SD_KIND_NORM_BETA, 0);
+    // q, k, v weights consecutive (each a multiple of 256 bytes): one [3C, C] matrix; same for the biases
+    a.qkv = tab.add("mid.attn.q.weight", {C, C}, SD_KIND_WEIGHT, C);
+    tab.add("mid.attn.k.weight", {C, C}, SD_KIND_WEIGHT, C);
+    tab.add("mid.attn.v.weight", {C, C}, SD_KIND_WEIGHT, C);
+    a.qkv_b = tab.add("mid.attn.q.bias", {C}, SD_KIND_BIAS, C);
+    tab.add("mid.attn.k.bias", {C}, SD_KIND_BIAS, C);
+    tab.add("mid.attn.v.bias", {C}, SD_KIND_BIAS, C);
+    a.ow = tab.add("mid.attn.out.weight", {C, C}, SD_KIND_WEIGHT, C);
+    a.ob = tab.add("mid.attn.out.bias", {C}, SD_KIND_BIAS, C);
+  }
+  v.mid_res1 = add_vae_resblock(tab, "mid.res.1", ch[0], ch[0]);
+  int c_prev = ch[0];
+  for (int i = 0; i < L; ++i) {
+    VaeW::Level lv;
+    lv.C = ch[i];
+    for (int j = 0; j <= cfg.layers_per_block; ++j) {
+      lv.res.push_back(add_vae_resblock(tab, "up." + std::to_string(i) + ".res." + std::to_string(j), c_prev, ch[i]));
+      c_prev = ch[i];
+    }
+    lv.has_up = i < L - 1;
+    if (lv.has_up) lv.up = add_conv3x3(tab, "up." + std::to_string(i) + ".up", ch[i], ch[i]);
+    v.up.push_back(lv);
+  }
+  v.out = add_output(tab, ch[L - 1], cfg.out_channels);
+  return v;
+}
+
 namespace {
 
 float bf16_to_f32(uint16_t b) {

@@ -125,6 +125,29 @@ struct UNetW {
 };
 UNetW add_unet(Table& tab, const sd_unet_cfg& cfg);
 
+// VAE decoder: resblocks without a time embedding (tw = tb = -1); the attention's
+// q/k/v weights are one [3C, C] matrix and their biases one [3C] vector.
+struct VaeAttnW {
+  int C;
+  int64_t ng, nb, qkv, qkv_b, ow, ob;
+};
+struct VaeW {
+  ConvW post_quant;  // 1x1, [lc][lc]
+  ConvW conv_in;
+  int conv_in_kp;
+  ResW mid_res0, mid_res1;
+  VaeAttnW mid_attn;
+  struct Level {
+    std::vector<ResW> res;
+    bool has_up;
+    ConvW up;
+    int C;
+  };
+  std::vector<Level> up;
+  OutW out;
+};
+VaeW add_vae(Table& tab, const sd_vae_cfg& cfg);
+
 int conv_in_kp(int c_in);
 
 // Canonical (host, BF16 bits) -> packed (host).

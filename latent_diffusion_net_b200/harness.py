@@ -51,6 +51,8 @@ class Module:
             self.rows, self.canon_n, self.packed_n = B.sd_transformer_weight_layout(cfg)
         elif kind == "unet":
             self.rows, self.canon_n, self.packed_n = B.sd_unet_weight_layout(cfg)
+        elif kind == "vae":
+            self.rows, self.canon_n, self.packed_n = B.sd_vae_weight_layout(cfg)
         else:
             raise ValueError(kind)
         self.packed_dev = None
@@ -69,6 +71,8 @@ class Module:
             return B.sd_resblock_pack_weights(self.cfg, canonical_u16, self.packed_n)
         if self.kind == "attn":
             return B.sd_transformer_pack_weights(self.cfg, canonical_u16, self.packed_n)
+        if self.kind == "vae":
+            return B.sd_vae_pack_weights(self.cfg, canonical_u16, self.packed_n)
         return B.sd_unet_pack_weights(self.cfg, canonical_u16, self.packed_n)
 
     def load(self, canonical_u16, device="cuda"):
@@ -81,6 +85,8 @@ class Module:
             self.ws_bytes = B.sd_resblock_workspace_size(self.cfg)
         elif self.kind == "attn":
             self.ws_bytes = B.sd_transformer_workspace_size(self.cfg)
+        elif self.kind == "vae":
+            self.ws_bytes = B.sd_vae_workspace_size(self.cfg)
         else:
             self.ws_bytes = B.sd_unet_workspace_size(self.cfg)
         self.ws = workspace(self.ws_bytes, device)
@@ -115,6 +121,9 @@ class Workload:
         if s["kind"] in ("unet", "denoise"):
             self.cfg = B.unet_cfg(height=s["H"], width=s["W"], **UNETS[s["unet"]])
             self.modules = [Module("unet", self.cfg)]
+        elif s["kind"] == "vae":
+            self.cfg = B.vae_cfg(s["H"], s["W"])
+            self.modules = [Module("vae", self.cfg)]
         else:
             self.modules.append(Module("time", B.time_cfg()))
             C, H, W = s["C"], s["H"], s["W"]
@@ -150,6 +159,9 @@ class Workload:
         if s["kind"] == "denoise":
             self.out = self.dev_inputs["x"]
             return
+        if s["kind"] == "vae":
+            self.out = torch.empty(64 * s["H"] * s["W"] * 3, dtype=torch.bfloat16, device=d)
+            return
         C, H, W = s["C"], s["H"], s["W"]
         self.temb = torch.empty(1280, dtype=torch.float32, device=d)
         self.bufs = [torch.empty(H * W * C, dtype=torch.bfloat16, device=d) for _ in range(2)]
@@ -166,6 +178,10 @@ class Workload:
         s = self.spec
         x = self.dev_inputs["x"] if latent is None else latent
         ctx = self.dev_inputs["ctx"] if context is None else context
+        if s["kind"] == "vae":
+            m = self.modules[0]
+            B.sd_vae_decode(self.cfg, m.packed_dev, x, self.out, m.ws, m.ws_bytes, stream)
+            return self.out
         if s["kind"] == "denoise":
             m = self.modules[0]
             B.sd_denoise(self.cfg, m.packed_dev, B.SD_SAMPLER_DDIM, self.alphas_cumprod, [s["timestep"]],
@@ -212,8 +228,10 @@ def make_inputs(wid):
         mask = synth.mask_rectangle(seed, H, W)[0].reshape(H, W, 1)
         out["x"] = np.concatenate([noisy, masked, mask], axis=2)
         out["text"] = synth.normal_bf16(seed, synth.IDX_TEXT, (UNETS[s["unet"]]["add_text_dim"],))
-    elif s["kind"] in ("unet", "denoise"):
+    elif s["kind"] in ("unet", "denoise", "vae"):
         out["x"] = synth.normal_bf16(seed, synth.IDX_X, (s["H"], s["W"], 4))
+        if s["kind"] == "vae":
+            return out  # the decoder has no context
     else:
         out["x"] = synth.normal_bf16(seed, synth.IDX_X, (s["H"], s["W"], s["C"]))
     out["ctx"] = synth.normal_bf16(seed, synth.IDX_CTX, (CTX_LEN, s["ctx_dim"]))
@@ -261,7 +279,33 @@ def flops(wid):
         return tm + res(hw, C, C) + tx(hw, C, s["depth"], s["ctx_dim"]) + conv(s["inpaint_hw"] ** 2, 9, 320)
     if s["kind"] == "denoise":
         return 2 * unet_flops(s["H"], s["W"], **UNETS[s["unet"]])
+    if s["kind"] == "vae":
+        return vae_flops(s["H"], s["W"])
     return unet_flops(s["H"], s["W"], **UNETS[s["unet"]])
+
+
+def vae_flops(H, W, latent_channels=4, out_channels=3, block_channels=(128, 256, 512, 512), layers_per_block=2):
+    """Algorithmic FLOPs of one VAE decode (2MNK per convolution and linear layer,
+    4 N^2 C for the single-head attention)."""
+    def conv(hw, ci, co, k=3):
+        return 2.0 * hw * co * ci * k * k
+
+    def res(hw, ci, co):
+        return conv(hw, ci, co) + conv(hw, co, co) + (conv(hw, ci, co, 1) if ci != co else 0.0)
+
+    ch = list(reversed(block_channels))
+    hw = H * W
+    f = conv(hw, latent_channels, latent_channels, 1) + conv(hw, latent_channels, ch[0])
+    f += 2 * res(hw, ch[0], ch[0]) + 4 * 2.0 * hw * ch[0] * ch[0] + 4.0 * hw * hw * ch[0]
+    c_prev = ch[0]
+    for i, c in enumerate(ch):
+        for _ in range(layers_per_block + 1):
+            f += res(hw, c_prev, c)
+            c_prev = c
+        if i < len(ch) - 1:
+            hw *= 4
+            f += conv(hw, c, c)
+    return f + conv(hw, ch[-1], out_channels)
 
 
 def unet_flops(H, W, in_channels, block_channels, attn_depth, mid_depth, ctx_dim, add_text_dim=0, add_time_ids=0,

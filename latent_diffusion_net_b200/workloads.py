@@ -31,6 +31,8 @@ timestep is 500. Activations are NHWC.
    with an unconditional context [77, 1024] ~ N(0, 1) (seed 4, stream 7), the
    guidance combination (scale 7.5) and a DDIM update at t = 500 on the page's
    linear schedule (0.0001 -> 0.02, 1000 steps).
+10. sd21_vae_decode_96: the VAE decoder on the 96x96 latent of workload 5's shape
+   (N(0, 1), seed 4) to a 768x768 RGB image; weights N(0, 1/fan_in), seed 6.
 """
 
 WORKLOADS = {
@@ -45,6 +47,7 @@ WORKLOADS = {
     8: dict(name="sd21_base_unet_step_128", seed=4, kind="unet", H=128, W=128, ctx_dim=1024, unet="sd21"),
     9: dict(name="sd21_base_guided_ddim_step_96", seed=4, kind="denoise", H=96, W=96, ctx_dim=1024, unet="sd21",
             guidance=7.5, timestep=500),
+    10: dict(name="sd21_vae_decode_96", seed=6, kind="vae", H=96, W=96),
 }
 
 # U-Net shapes (SD2.1 architecture page section 3; SDXL-Inpainting architecture

@@ -157,20 +157,37 @@ def vae_attention(x, params, prefix, groups=32, eps=1e-5):
     return x + o.T.reshape(C, H, W)
 
 
-def vae_decode(z, params, cfg: VAEConfig = SD_VAE):
-    """Latent z [latent_channels, h, w] -> image [out_channels, 8h, 8w]."""
+def vae_stages(z, params, cfg: VAEConfig = SD_VAE):
+    """The decode as a sequence of modules: yields (name, output) after the input
+    convolutions, each resblock, the attention, each upsampling conv and the
+    output head ("out", the image)."""
     z = np.asarray(z, dtype=np.float64) / cfg.scaling_factor
     G, eps = cfg.groups, cfg.eps
     h = conv2d(z, _w(params, "post_quant_conv.weight"), _w(params, "post_quant_conv.bias"), 1, 0)
     h = conv2d(h, _w(params, "conv_in.weight"), _w(params, "conv_in.bias"), 1, 1)
+    yield "conv_in", h
     h = vae_resblock(h, params, "mid.res.0", G, eps)
+    yield "mid.res.0", h
     h = vae_attention(h, params, "mid.attn", G, eps)
+    yield "mid.attn", h
     h = vae_resblock(h, params, "mid.res.1", G, eps)
+    yield "mid.res.1", h
     n = len(cfg.block_channels)
     for i in range(n):
         for j in range(cfg.layers_per_block + 1):
             h = vae_resblock(h, params, f"up.{i}.res.{j}", G, eps)
+            yield f"up.{i}.res.{j}", h
         if i < n - 1:
             h = conv2d(upsample_nearest2x(h), _w(params, f"up.{i}.up.weight"), _w(params, f"up.{i}.up.bias"), 1, 1)
+            yield f"up.{i}.up", h
     h = silu(group_norm(h, _w(params, "out.norm.gamma"), _w(params, "out.norm.beta"), G, eps))
-    return conv2d(h, _w(params, "conv_out.weight"), _w(params, "conv_out.bias"), 1, 1)
+    yield "out", conv2d(h, _w(params, "conv_out.weight"), _w(params, "conv_out.bias"), 1, 1)
+
+
+def vae_decode(z, params, cfg: VAEConfig = SD_VAE):
+    """Latent z [latent_channels, h, w] -> image [out_channels, 8h, 8w]: the
+    modules of ``vae_stages`` in order."""
+    out = None
+    for _, out in vae_stages(z, params, cfg):
+        pass
+    return out

@@ -227,3 +227,15 @@ def test_conditioned_step_and_hooks_validate_on_host():
     B.sd_record_begin(fake, 0)
     assert B.sd_record_end() == (0, 0)
     assert B.sd_record_read() == []
+
+
+def test_vae_table_matches_oracle_and_validates():
+    from oracle import vae
+    rows, canon, packed = B.sd_vae_weight_layout(B.vae_cfg(96, 96))
+    assert strip(rows, "") == oracle_rows(vae.enumerate_vae_decoder_params(), "")
+    assert canon == 49_490_199
+    assert B.sd_vae_workspace_size(B.vae_cfg(96, 96)) > B.sd_vae_workspace_size(B.vae_cfg(32, 32)) > 0
+    fake = 1 << 20
+    assert B.sd_vae_decode(B.vae_cfg(10, 10), fake, fake, fake, fake, 10 ** 10, check=False) == 3  # 100 tokens
+    assert B.sd_vae_decode(B.vae_cfg(16, 16, groups=64), fake, fake, fake, fake, 10 ** 10, check=False) == 3
+    assert B.sd_vae_decode(B.vae_cfg(16, 16), fake, None, fake, fake, 10 ** 10, check=False) == 1

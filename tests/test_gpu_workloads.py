@@ -54,12 +54,16 @@ def make_workload(wid):
     return wl
 
 
+def workload_params(wid, wl):
+    params = {}
+    for r, canon in zip(oracle_rows_for(wid), wl.canonical):
+        params.update(oracle_params(r, canon))
+    return params
+
+
 def oracle_forward(wid, wl, record=None):
     s = WORKLOADS[wid]
-    rows = oracle_rows_for(wid)
-    params = {}
-    for r, canon in zip(rows, wl.canonical):
-        params.update(oracle_params(r, canon))
+    params = workload_params(wid, wl)
     inp = wl.inputs
     if s["kind"] == "unet":
         cfg = UNET_CFGS[s["unet"]]
