@@ -53,10 +53,11 @@ sd_status device_info(DevInfo* out) {
 
 // ------------------------------------------------------------------ workspace arena
 constexpr size_t kHeaderBytes = 256;   // word 0: device error flags
-constexpr int kMaxGnLaunches = 256;      // GroupNorm statistics slots per call
+constexpr int kMaxGnLaunches = 128;      // GroupNorm statistics slots per call
 constexpr int kMaxGroups = 64;
-// per GroupNorm launch: 2 * kMaxGroups sums, then the barrier counter of the single-pass kernel (padded)
-constexpr int kGnSlotWords = 2 * kMaxGroups + 2;
+// per GroupNorm launch: one 128-byte line of sums per group, then a line holding
+// the barrier counter of the single-pass kernel
+constexpr int kGnSlotWords = sdk::kGnAccStride * kMaxGroups + 16;
 constexpr size_t kGnAccBytes = (size_t)kMaxGnLaunches * kGnSlotWords * sizeof(unsigned long long);
 constexpr int kMaxStatBlocks = 512;  // GroupNorm partial-sum slots: 2 CTAs per SM, up to 256 SMs
 
@@ -143,7 +144,7 @@ sd_status run_gn(const Ctx& c, const bf16* x0, int C0, const bf16* x1, int C1, i
                  const bf16* gamma, const bf16* beta, int silu, bf16* y) {
   if (!c.gn_seq || *c.gn_seq >= kMaxGnLaunches) return SD_ERR_UNSUPPORTED;
   unsigned long long* acc = c.gn_acc + (size_t)(*c.gn_seq)++ * kGnSlotWords;
-  unsigned int* counter = reinterpret_cast<unsigned int*>(acc + 2 * kMaxGroups);
+  unsigned int* counter = reinterpret_cast<unsigned int*>(acc + sdk::kGnAccStride * kMaxGroups);
   const int nk = sdk::groupnorm_plan_launches(C0 + C1, HW, c.sms);
   // algorithmic bytes: read once and write once (the two-kernel form reads twice)
   sdp::Scope sc("groupnorm", sdp::F_GN_APPLY, 0, (nk == 1 ? 2.0 : 3.0) * HW * (C0 + C1) * 2, c.st, nk);

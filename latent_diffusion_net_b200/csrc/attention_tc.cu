@@ -20,8 +20,7 @@
 //              log2 domain, and forms P = exp2(s*log2e/8 - m) two at a time: the
 //              pair of FP32 exponents is rounded to FP16 and one packed
 //              ex2.approx.f16x2 gives both probabilities, already in the FP16
-//              form the PV product takes (so one exponential-unit issue serves
-//              two keys and no conversion follows). P goes to shared memory (the
+//              form the PV product takes. P goes to shared memory (the
 //              A operand of the PV product, 128-byte swizzled); the row sum is
 //              kept in four packed FP16 partial sums per tile, added into FP32
 //              once per tile. The output O lives in TMEM and is rescaled only
@@ -238,6 +237,13 @@ __global__ void __launch_bounds__(192, 2)
     mbar_init(q_empty, 1);
     *abort_flag = 0;
     fence_barrier_init();
+    // descriptors and arguments are kernel parameters: fetch them into the caches
+    // before waiting for the previous kernel
+    tma_prefetch_desc(&maps.q);
+    tma_prefetch_desc(&maps.kv);
+    const int64_t touch = args.steps + args.ctas + args.qtiles + args.ktiles + args.Nq + args.Nk + args.q_col +
+                          args.k_col + args.v_col;
+    asm volatile("" ::"l"(touch));
   }
   if (warp == 5) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -252,8 +258,6 @@ __global__ void __launch_bounds__(192, 2)
   if (warp == 4) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&maps.q);
-      tma_prefetch_desc(&maps.kv);
       int ii = 0;  // items started
       int X = (int)(w0 / nt), j = (int)(w0 % nt);
       for (int t = 0; t < T; ++t, j = (j + 1 == nt) ? 0 : j + 1, X += (j == 0)) {

@@ -176,6 +176,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     mbar_init(hold_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
+    // the tensor maps are kernel parameters, not data of the previous kernel: fetch
+    // them into the descriptor cache while that kernel is still running
+    for (int i = 0; i < kGemmMaxA; ++i) {
+      tma_prefetch_desc(&maps.a[i]);
+      tma_prefetch_desc(&maps.at[i]);
+    }
+    tma_prefetch_desc(&maps.b[0]);
+    tma_prefetch_desc(&maps.b[1]);
+    // touch the parameters the producer and MMA loops read before their first
+    // load and MMA, so that their constant-cache misses also fall before the wait
+    int touch = args.units + args.splits + args.tiles_n + args.tiles_x + args.tiles_m + args.BH + args.BW +
+                args.kb_per_split + args.total_kb + args.nseg + args.a_bytes;
+#pragma unroll
+    for (int i = 0; i < kGemmMaxSeg; ++i) touch += args.seg[i].amap + args.seg[i].per + args.seg[i].bstep;
+    asm volatile("" ::"r"(touch));
   }
   if (warp == 1) tmem_alloc_2sm(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -202,12 +217,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     if (lane == 0 && !*abort_flag) {
-      for (int i = 0; i < kGemmMaxA; ++i) {
-        tma_prefetch_desc(&maps.a[i]);
-        tma_prefetch_desc(&maps.at[i]);
-      }
-      tma_prefetch_desc(&maps.b[0]);
-      tma_prefetch_desc(&maps.b[1]);
       const uint32_t tall_bytes = (uint32_t)((args.BH + 2) * args.BW * kBK * 2 + 3 * kBTileBytes);
       const uint32_t single_bytes = (uint32_t)(kATileBytes + kBTileBytes);
       uint32_t q = 0;        // stages issued by this CTA so far

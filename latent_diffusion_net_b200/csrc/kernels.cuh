@@ -7,9 +7,15 @@
 
 namespace sdk {
 
+// GroupNorm statistics accumulators: group g's fixed-point sum and sum of squares
+// are words kGnAccStride*g and kGnAccStride*g + 1, so every group has a 128-byte
+// line of its own (the atomics of all CTAs on one group do not queue behind
+// those of the other groups).
+constexpr int kGnAccStride = 16;
+
 // GroupNorm (+SiLU) of the channel concatenation [x0 | x1] (x1 may be null with
-// C1 = 0) into y. `acc` holds 2*G and `counter` one zero-initialised word used
-// by this call only. When each CTA's share of the pixels fits in shared memory
+// C1 = 0) into y. `acc` holds kGnAccStride*G zero-initialised words and `counter`
+// one zero-initialised word used by this call only. When each CTA's share of the pixels fits in shared memory
 // one kernel does both passes (statistics, grid barrier, normalisation; a
 // barrier that times out raises ERR_MBAR_TIMEOUT in *err); otherwise a
 // statistics kernel and an apply kernel run (counter / err may then be null).

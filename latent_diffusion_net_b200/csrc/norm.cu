@@ -32,6 +32,16 @@ __device__ __forceinline__ long long to_fixed(float v, double scale) {
   return __double2ll_rn(d);
 }
 
+// SiLU(x) = x * sigmoid(x) = h + h * tanh(h) with h = x / 2: one MUFU operation
+// (tanh.approx, relative error about 2^-11) instead of an exponential and a
+// reciprocal; the normalise + SiLU pass is bound by that unit.
+__device__ __forceinline__ float silu_tanh(float x) {
+  const float h = 0.5f * x;
+  float th;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(h));
+  return fmaf(h, th, h);
+}
+
 __global__ void gn_stats_kernel(const __nv_bfloat16* __restrict__ x0, int C0, const __nv_bfloat16* __restrict__ x1,
                                 int C1, int HW, int G, int ppi, unsigned long long* __restrict__ acc) {
   extern __shared__ float4 red[];  // [blockDim.x]
@@ -106,8 +116,8 @@ __global__ void gn_stats_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
         }
       }
     }
-    atomicAdd(&acc[2 * g], (unsigned long long)to_fixed(s, kSumScale));
-    atomicAdd(&acc[2 * g + 1], (unsigned long long)to_fixed(q, kSqScale));
+    atomicAdd(&acc[kGnAccStride * g], (unsigned long long)to_fixed(s, kSumScale));
+    atomicAdd(&acc[kGnAccStride * g + 1], (unsigned long long)to_fixed(q, kSqScale));
   }
 }
 
@@ -123,8 +133,8 @@ __global__ void gn_apply_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
   const int cpg = C / G;
   if (threadIdx.x < G) {
     const double cnt = (double)HW * cpg;
-    const double mean = (double)(long long)acc[2 * threadIdx.x] / kSumScale / cnt;
-    double var = (double)(long long)acc[2 * threadIdx.x + 1] / kSqScale / cnt - mean * mean;
+    const double mean = (double)(long long)acc[kGnAccStride * threadIdx.x] / kSumScale / cnt;
+    double var = (double)(long long)acc[kGnAccStride * threadIdx.x + 1] / kSqScale / cnt - mean * mean;
     if (var < 0.0) var = 0.0;
     gstat[threadIdx.x] = make_float2((float)mean, (float)(1.0 / sqrt(var + (double)eps)));
   }
@@ -137,39 +147,67 @@ __global__ void gn_apply_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
   __syncthreads();
   const int V = C >> 3;
   const size_t total = (size_t)HW * V;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  auto src_of = [&](size_t i) {
     const int p = (int)(i / V);
     const int c = (int)(i % V) * 8;
-    const __nv_bfloat16* src = (c < C0) ? (x0 + (size_t)p * C0 + c) : (x1 + (size_t)p * C1 + (c - C0));
-    const uint4 w = *reinterpret_cast<const uint4*>(src);
+    return (c < C0) ? (x0 + (size_t)p * C0 + c) : (x1 + (size_t)p * C1 + (c - C0));
+  };
+  auto apply = [&](size_t i, const uint4 w) {
+    const int p = (int)(i / V);
+    const int c = (int)(i % V) * 8;
     float f[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
                   bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float2 s = ab[c + j];
       float o = fmaf(f[j], s.x, s.y);
-      if (silu) o = __fdividef(o, 1.0f + __expf(-o));
+      if (silu) o = silu_tanh(o);
       f[j] = o;
     }
     *reinterpret_cast<uint4*>(y + (size_t)p * C + c) =
         make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+  };
+  size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  // four independent loads in flight per thread before any is used
+  for (; i + 3 * stride < total; i += 4 * stride) {
+    uint4 w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) w[u] = __ldcs(reinterpret_cast<const uint4*>(src_of(i + u * stride)));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) apply(i + u * stride, w[u]);
   }
+  for (; i < total; i += stride) apply(i, __ldcs(reinterpret_cast<const uint4*>(src_of(i))));
 }
 
-// Single-pass GroupNorm: every CTA copies its contiguous pixel range of [x0 | x1]
-// into shared memory while summing it (the statistics of gn_stats_kernel, same
-// fixed-point accumulators), then all CTAs meet at a grid-wide barrier (an
-// arrival counter polled with a bounded wait), read the final sums and
-// normalise their shared-memory copy. The tensor is read once and written once,
-// in one launch. The grid never exceeds the CTAs that can be resident at once:
+// Single-pass GroupNorm. Every CTA loads its contiguous pixel range of [x0 | x1]
+// in one burst (each thread holds up to kGnPx 16-byte vectors of one 8-channel
+// column, all requested before any is used, then parked in shared memory), adds
+// their sums and sums of squares per group as 64-bit fixed point (shared-memory
+// integer atomics, then one global atomic per group and CTA on the group's own
+// 128-byte line: integer addition, so the totals do not depend on arrival
+// order), meets the other CTAs at a grid-wide barrier (an arrival counter polled
+// with a bounded wait), and normalises the values it holds. The tensor is read
+// once and written once, in one launch. Each thread keeps the same 8 channels
+// throughout, so it fetches their gamma and beta (weights, not data of the
+// previous kernel) before waiting for that kernel, and forms its own scale and
+// shift from the two groups' statistics. The grid never exceeds one CTA per SM:
 // each CTA waits in griddepcontrol.wait for the previous kernel, which then
 // leaves the whole GPU to this grid, and this kernel lets its dependents launch
-// only after the barrier, so every CTA is resident before any waits on the others.
-__global__ void gn_fused_kernel(const __nv_bfloat16* __restrict__ x0, int C0, const __nv_bfloat16* __restrict__ x1,
-                                int C1, int HW, int G, int ppi, float eps, const __nv_bfloat16* __restrict__ gamma,
-                                const __nv_bfloat16* __restrict__ beta, int silu, __nv_bfloat16* __restrict__ y,
-                                unsigned long long* __restrict__ acc, unsigned int* counter, int* err) {
-  extern __shared__ __align__(16) uint8_t gsm[];
+// only after the barrier, so every CTA is resident before any waits on the
+// others.
+constexpr int kGnPx = 8;          // pixels held per thread
+constexpr int kGnThreads = 1024;  // at most; V * ppi threads with ppi = kGnThreads / V
+constexpr int kGnMaxV = 320;      // 8-channel columns (C <= 2560)
+
+__global__ void __launch_bounds__(kGnThreads, 1)
+    gn_fused_kernel(const __nv_bfloat16* __restrict__ x0, int C0, const __nv_bfloat16* __restrict__ x1, int C1,
+                    int HW, int G, int ppi, int chunk, float eps, const __nv_bfloat16* __restrict__ gamma,
+                    const __nv_bfloat16* __restrict__ beta, int silu, __nv_bfloat16* __restrict__ y,
+                    unsigned long long* __restrict__ acc, unsigned int* counter, int* err) {
+  extern __shared__ __align__(16) uint4 slice[];  // [kGnPx][blockDim.x], then red [blockDim.x] float4
+  float4* red = reinterpret_cast<float4*>(slice + kGnPx * blockDim.x);
+  __shared__ float4 col[kGnMaxV];  // per 8-channel column: sums of its two groups' parts
   __shared__ float2 gstat[64];
   __shared__ int give_up;
   const int C = C0 + C1;
@@ -179,14 +217,13 @@ __global__ void gn_fused_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
   const int v = t % V;
   const int pi = t / V;
   const int c = v * 8;
-  const int chunk = (HW + gridDim.x - 1) / gridDim.x;
   const int p0 = blockIdx.x * chunk;
   const int p1 = min(HW, p0 + chunk);
-  float4* red = reinterpret_cast<float4*>(gsm);                                   // [blockDim.x]
-  uint4* slice = reinterpret_cast<uint4*>(gsm + (size_t)blockDim.x * sizeof(float4));  // [chunk][V]
+  const uint4 gq = __ldg(reinterpret_cast<const uint4*>(gamma + c));
+  const uint4 bq = __ldg(reinterpret_cast<const uint4*>(beta + c));
+  if (t == 0) give_up = 0;
+  __syncthreads();
   pdl_wait();
-  const int ga = c / cpg;
-  const int split = (ga + 1) * cpg - c;  // channels c .. c+split-1 belong to ga, the rest to ga+1
   const __nv_bfloat16* base;
   int ld;
   if (c < C0) {
@@ -196,62 +233,68 @@ __global__ void gn_fused_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
     base = x1 + (c - C0);
     ld = C1;
   }
+  const bool active = pi < ppi;
+  // this thread's pixels p0 + pi + k*ppi, k < npx: one 16-byte vector each, all requested first
+  const int npx = active && p0 + pi < p1 ? (p1 - p0 - pi + ppi - 1) / ppi : 0;
+  const uint4* q = reinterpret_cast<const uint4*>(base + (size_t)(p0 + pi) * ld);
+  const int qstep = ppi * ld / 8;
+  uint4 w[kGnPx];
+#pragma unroll
+  for (int k = 0; k < kGnPx; ++k) w[k] = k < npx ? __ldcg(q + k * qstep) : make_uint4(0, 0, 0, 0);
+  // kept in shared memory across the barrier (registers stay free for the statistics)
+#pragma unroll
+  for (int k = 0; k < kGnPx; ++k)
+    if (k < npx) slice[k * blockDim.x + t] = w[k];
+  const int ga = c / cpg;
+  const int split = (ga + 1) * cpg - c;  // channels c .. c+split-1 belong to ga, the rest to ga+1
   float sa = 0.f, qa = 0.f, sb = 0.f, qb = 0.f;
-  auto accum = [&](const uint4 w) {
-    const float f[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
-                        bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+#pragma unroll
+  for (int k = 0; k < kGnPx; ++k) {
+    if (k >= npx) break;
+    const uint32_t u[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (j < split) {
-        sa += f[j];
-        qa = fmaf(f[j], f[j], qa);
-      } else {
-        sb += f[j];
-        qb = fmaf(f[j], f[j], qb);
-      }
-    }
-  };
-  if (pi < ppi) {
-    // four independent loads in flight per thread before any is used
-    int p = p0 + pi;
-    for (; p + 3 * ppi < p1; p += 4 * ppi) {
-      uint4 w[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) w[u] = __ldcg(reinterpret_cast<const uint4*>(base + (size_t)(p + u * ppi) * ld));
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        slice[(size_t)(p + u * ppi - p0) * V + v] = w[u];
-        accum(w[u]);
-      }
-    }
-    for (; p < p1; p += ppi) {
-      const uint4 w = __ldcg(reinterpret_cast<const uint4*>(base + (size_t)p * ld));
-      slice[(size_t)(p - p0) * V + v] = w;
-      accum(w);
+      const float f = (j & 1) ? bf16hi(u[j >> 1]) : bf16lo(u[j >> 1]);
+      const bool in_a = j < split;
+      sa += in_a ? f : 0.f;
+      qa = fmaf(in_a ? f : 0.f, f, qa);
+      sb += in_a ? 0.f : f;
+      qb = fmaf(in_a ? 0.f : f, f, qb);
     }
   }
-  red[t] = make_float4(sa, qa, sb, qb);
-  if (t == 0) give_up = 0;
+  // CTA reduction in a fixed order (FP32, the same bits every run): the rows of each
+  // 8-channel column, then the one to three columns of each group; one global
+  // fixed-point atomic per group and CTA
+  red[t] = active ? make_float4(sa, qa, sb, qb) : make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  if (t < V) {
+    float4 r = red[t];
+    for (int pp = 1; pp < ppi; ++pp) {
+      const float4 o = red[pp * V + t];
+      r.x += o.x;
+      r.y += o.y;
+      r.z += o.z;
+      r.w += o.w;
+    }
+    col[t] = r;
+  }
   __syncthreads();
   if (t < G) {
-    const int g = t;
-    const int vlo = (g * cpg) / 8;
-    const int vhi = min(V - 1, ((g + 1) * cpg - 1) / 8);
-    float s = 0.f, q = 0.f;
-    for (int pp = 0; pp < ppi; ++pp) {
-      for (int vv = vlo; vv <= vhi; ++vv) {
-        const float4 r = red[pp * V + vv];
-        if ((vv * 8) / cpg == g) {
-          s += r.x;
-          q += r.y;
-        } else {
-          s += r.z;
-          q += r.w;
-        }
+    const int vlo = (t * cpg) / 8;
+    const int vhi = min(V - 1, ((t + 1) * cpg - 1) / 8);
+    float s = 0.f, q2 = 0.f;
+    for (int vv = vlo; vv <= vhi; ++vv) {
+      const float4 r = col[vv];
+      if ((vv * 8) / cpg == t) {  // the column's first channels belong to group t
+        s += r.x;
+        q2 += r.y;
+      } else {
+        s += r.z;
+        q2 += r.w;
       }
     }
-    atomicAdd(&acc[2 * g], (unsigned long long)to_fixed(s, kSumScale));
-    atomicAdd(&acc[2 * g + 1], (unsigned long long)to_fixed(q, kSqScale));
+    atomicAdd(&acc[kGnAccStride * t], (unsigned long long)to_fixed(s, kSumScale));
+    atomicAdd(&acc[kGnAccStride * t + 1], (unsigned long long)to_fixed(q2, kSqScale));
   }
   __syncthreads();
   if (t == 0) {
@@ -263,7 +306,7 @@ __global__ void gn_fused_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
     do {
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(counter) : "memory");
       if (seen >= gridDim.x) break;
-      __nanosleep(64);
+      __nanosleep(32);
     } while (++n < kSpinLimit);
     if (seen < gridDim.x) {
       give_up = 1;
@@ -275,80 +318,89 @@ __global__ void gn_fused_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
   if (give_up) return;
   if (t < G) {
     const double cnt = (double)HW * cpg;
-    const double mean = (double)(long long)__ldcg(&acc[2 * t]) / kSumScale / cnt;
-    double var = (double)(long long)__ldcg(&acc[2 * t + 1]) / kSqScale / cnt - mean * mean;
+    const double mean = (double)(long long)__ldcg(&acc[kGnAccStride * t]) / kSumScale / cnt;
+    double var = (double)(long long)__ldcg(&acc[kGnAccStride * t + 1]) / kSqScale / cnt - mean * mean;
     if (var < 0.0) var = 0.0;
     gstat[t] = make_float2((float)mean, (float)(1.0 / sqrt(var + (double)eps)));
   }
   __syncthreads();
-  if (pi >= ppi) return;
-  float a[8], b[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float2 stt = gstat[(c + j) / cpg];
-    a[j] = stt.y * __bfloat162float(gamma[c + j]);
-    b[j] = __bfloat162float(beta[c + j]) - stt.x * a[j];
-  }
-  for (int p = p0 + pi; p < p1; p += ppi) {
-    const uint4 w = slice[(size_t)(p - p0) * V + v];
-    float f[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
-                  bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+  if (!active) return;
+  // this thread's 8 channels: scale a = rstd * gamma, shift b = beta - mean * a
+  float sc[8], sh[8];
+  {
+    const uint32_t gu[4] = {gq.x, gq.y, gq.z, gq.w};
+    const uint32_t bu[4] = {bq.x, bq.y, bq.z, bq.w};
+    const float2 st_a = gstat[ga];
+    const float2 st_b = split < 8 ? gstat[ga + 1] : st_a;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      float o = fmaf(f[j], a[j], b[j]);
-      if (silu) o = __fdividef(o, 1.0f + __expf(-o));
+      const float2 st = j < split ? st_a : st_b;
+      const float gj = (j & 1) ? bf16hi(gu[j >> 1]) : bf16lo(gu[j >> 1]);
+      const float bj = (j & 1) ? bf16hi(bu[j >> 1]) : bf16lo(bu[j >> 1]);
+      sc[j] = st.y * gj;
+      sh[j] = bj - st.x * sc[j];
+    }
+  }
+  __nv_bfloat16* yq = y + (size_t)(p0 + pi) * C + c;
+#pragma unroll
+  for (int k = 0; k < kGnPx; ++k) {
+    if (k >= npx) break;
+    const uint4 wk = slice[k * blockDim.x + t];
+    float f[8] = {bf16lo(wk.x), bf16hi(wk.x), bf16lo(wk.y), bf16hi(wk.y),
+                  bf16lo(wk.z), bf16hi(wk.z), bf16lo(wk.w), bf16hi(wk.w)};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float o = fmaf(f[j], sc[j], sh[j]);
+      if (silu) o = silu_tanh(o);
       f[j] = o;
     }
-    *reinterpret_cast<uint4*>(y + (size_t)p * C + c) =
+    *reinterpret_cast<uint4*>(yq + (size_t)k * ppi * C) =
         make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
   }
 }
 
-constexpr int kFusedSmemLimit = 200 * 1024;
-
-// Pixels handled side by side by one CTA of the single-pass kernel: as many as
-// keep the CTA at most 1024 threads, so that each SM has many loads in flight.
-static int fused_ppi(int V) { return V >= 1024 ? 1 : 1024 / V; }
-
-static size_t fused_smem(int C, int HW, int num_sms) {
+// Geometry of the single-pass kernel for [HW, C]: CTAs, pixels per CTA, threads
+// per pixel row; false when the tensor does not fit in the registers of one
+// wave of CTAs.
+static bool fused_plan(int C, int HW, int num_sms, int* nblk, int* chunk, int* ppi) {
   const int V = C / 8;
-  const int chunk = (HW + num_sms - 1) / num_sms;
-  return (size_t)V * fused_ppi(V) * sizeof(float4) + (size_t)chunk * C * 2;
+  if (V > kGnMaxV) return false;
+  *ppi = kGnThreads / V;
+  int n = num_sms;
+  int ch = (HW + n - 1) / n;
+  if (ch > kGnPx * *ppi) return false;
+  *nblk = (HW + ch - 1) / ch;  // no CTA without pixels
+  *chunk = ch;
+  return true;
 }
 
 int groupnorm_plan_launches(int C, int HW, int num_sms) {
-  return fused_smem(C, HW, num_sms) <= (size_t)kFusedSmemLimit ? 1 : 2;
+  int a, b, c;
+  return fused_plan(C, HW, num_sms, &a, &b, &c) ? 1 : 2;
 }
 
 int launch_groupnorm(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, int C1, int HW, int G, float eps,
                      const __nv_bfloat16* gamma, const __nv_bfloat16* beta, int silu, __nv_bfloat16* y,
                      unsigned long long* acc, unsigned int* counter, int num_sms, cudaStream_t st, int* err) {
+  // 8-channel vectors never straddle the two sources, and one vector spans at most two groups
+  if (C0 % 8 || C1 % 8 || G < 1 || (C0 + C1) % G) return -1;
+  const int cpg = (C0 + C1) / G;
+  if (cpg < 8 && cpg != 4) return -1;
   {
-    // single pass when every CTA's pixel range fits in shared memory
-    const int C = C0 + C1;
-    const int V = C / 8;
-    const int ppi = fused_ppi(V);
-    const int threads = V * ppi;
-    if (threads < G || threads > 1024 || G > 64) return -1;
-    static bool attr_set = false;  // benign race: the attribute value is identical for every caller
-    int nblk = num_sms;
-    const size_t smem = fused_smem(C, HW, num_sms);
-    if (counter && err && smem <= (size_t)kFusedSmemLimit) {
+    // single pass when every CTA's pixel range fits in its threads' registers
+    int nblk, chunk, ppi;
+    if (counter && err && G <= 64 && fused_plan(C0 + C1, HW, num_sms, &nblk, &chunk, &ppi)) {
+      const int threads = (C0 + C1) / 8 * ppi;
+      const size_t smem = (size_t)(kGnPx + 1) * threads * sizeof(uint4);
+      static bool attr_set = false;  // benign race: the attribute value is identical for every caller
       if (!attr_set) {
-        if (cudaFuncSetAttribute(gn_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmemLimit) !=
-            cudaSuccess)
-          return (int)cudaGetLastError();
+        const cudaError_t e = cudaFuncSetAttribute(gn_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)((size_t)(kGnPx + 1) * kGnThreads * sizeof(uint4)));
+        if (e != cudaSuccess) return (int)e;
         attr_set = true;
       }
-      int occ = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gn_fused_kernel, threads, smem) == cudaSuccess &&
-          occ >= 1) {
-        const int chunk_n = (HW + nblk - 1) / nblk;
-        nblk = (HW + chunk_n - 1) / chunk_n;  // no CTA without pixels
-        return (int)launch_pdl(gn_fused_kernel, dim3(nblk), dim3(threads), smem, st, x0, C0, x1, C1, HW, G, ppi, eps,
-                               gamma, beta, silu, y, acc, counter, err);
-      }
-      (void)cudaGetLastError();
+      return (int)launch_pdl(gn_fused_kernel, dim3(nblk), dim3(threads), smem, st, x0, C0, x1, C1, HW, G, ppi, chunk,
+                             eps, gamma, beta, silu, y, acc, counter, err);
     }
   }
   const int C = C0 + C1;
@@ -358,13 +410,13 @@ int launch_groupnorm(const __nv_bfloat16* x0, int C0, const __nv_bfloat16* x1, i
   if (threads < G || threads > 1024 || G > 64) return -1;
   int nblk = HW / (ppi * 8);  // about 8 pixels per thread
   if (nblk < 1) nblk = 1;
-  if (nblk > 2 * num_sms) nblk = 2 * num_sms;
+  if (nblk > 4 * num_sms) nblk = 4 * num_sms;
   cudaError_t e = launch_pdl(gn_stats_kernel, dim3(nblk), dim3(threads), threads * sizeof(float4), st, x0, C0, x1, C1,
                              HW, G, ppi, acc);
   if (e != cudaSuccess) return (int)e;
   const size_t total = (size_t)HW * V;
   int blocks = (int)((total + 255) / 256);
-  if (blocks > 2 * num_sms) blocks = 2 * num_sms;
+  if (blocks > 8 * num_sms) blocks = 8 * num_sms;
   return (int)launch_pdl(gn_apply_kernel, dim3(blocks), dim3(256), C * sizeof(float2), st, x0, C0, x1, C1, HW, G, eps,
                          (const unsigned long long*)acc, gamma, beta, silu, y);
 }

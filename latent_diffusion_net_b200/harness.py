@@ -177,7 +177,7 @@ class Workload:
         """Enqueue one pass of the workload on ``stream``; returns the output tensor."""
         s = self.spec
         x = self.dev_inputs["x"] if latent is None else latent
-        ctx = self.dev_inputs["ctx"] if context is None else context
+        ctx = self.dev_inputs.get("ctx") if context is None else context
         if s["kind"] == "vae":
             m = self.modules[0]
             B.sd_vae_decode(self.cfg, m.packed_dev, x, self.out, m.ws, m.ws_bytes, stream)

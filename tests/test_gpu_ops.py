@@ -88,15 +88,24 @@ def test_downsample_conv(H, W, C):
     assert_close(dev_np(y, (H // 2, W // 2, C)), ref, OP_TOL)
 
 
-@pytest.mark.parametrize("H,W,C", [(20, 20, 320), (96, 96, 320)])
+# (176, 176, 320) and (96, 160, 640) hold more pixels per CTA than the single-pass
+# GroupNorm keeps on chip (8 per thread on 148 SMs), so they take the statistics +
+# apply kernel pair; the smaller ones take the single-pass kernel.
+@pytest.mark.parametrize("H,W,C", [(20, 20, 320), (96, 96, 320), (176, 176, 320), (96, 160, 640)])
 def test_output_head(H, W, C):
     rows = [("out.norm.gamma", (C,), "norm_gamma", 0), ("out.norm.beta", (C,), "norm_beta", 0)] + \
         model.enumerate_conv_params("conv_out", C, 4)
     m, p = load_module("conv", B.conv_cfg(H, W, C, 4), 15, rows, B.SD_CONV_OUTPUT, affine=True)
     x = synth.normal_bf16(15, 0, (H, W, C))
     y = torch.empty(H * W * 4, dtype=torch.bfloat16, device="cuda")
+    B.sd_profile_begin()
     B.sd_conv_fwd(m.cfg, B.SD_CONV_OUTPUT, m.packed_dev, Hn.to_dev_bf16(x), None, None, y, m.ws, m.ws_bytes)
+    B.sd_profile_end()
     torch.cuda.synchronize()
+    gn = [r for r in B.sd_profile_read() if r["kernel"] == "groupnorm"]
+    single_pass = H * W <= 148 * 8 * (1024 // (C // 8))
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert [r["kernels"] for r in gn] == [1 if single_pass else 2]
     g = oracle.silu(oracle.group_norm(chw(x), p["out.norm.gamma"], p["out.norm.beta"], 32, 1e-5))
     ref = hwc(oracle.conv2d(g, p["conv_out.weight"], p["conv_out.bias"], 1, 1))
     assert_close(dev_np(y, (H, W, 4)), ref, OP_TOL)
