@@ -197,15 +197,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // everything above touched only shared memory and TMEM: wait for the previous kernel here
-  pdl_wait();
-  pdl_trigger();
-  if (args.epi.rowstat_clear) {
-    // every kernel before this one has finished: the buffer's last reader among them
-    const int64_t n2 = args.epi.rowstat_clear_elems / 2;
-    ulonglong2* z = reinterpret_cast<ulonglong2*>(args.epi.rowstat_clear);
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += (int64_t)gridDim.x * blockDim.x)
-      z[i] = make_ulonglong2(0ull, 0ull);
+  // Everything above touched only shared memory and TMEM: wait for the previous
+  // kernel here. The producer thread (warp 0, lane 0) waits later, just before
+  // its first load, so that the setup of its first stage overlaps that kernel too.
+  auto after_wait = [&]() {
+    pdl_trigger();
+    if (args.epi.rowstat_clear) {
+      // every kernel before this one has finished: the buffer's last reader among them
+      const int64_t n2 = args.epi.rowstat_clear_elems / 2;
+      ulonglong2* z = reinterpret_cast<ulonglong2*>(args.epi.rowstat_clear);
+      for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += (int64_t)gridDim.x * blockDim.x)
+        z[i] = make_ulonglong2(0ull, 0ull);
+    }
+  };
+  if (threadIdx.x != 0) {
+    pdl_wait();
+    after_wait();
   }
   if (args.hold_spins > 0) {
     // timeout test: nothing ever arrives on hold_bar, so this bounded wait gives
@@ -216,6 +223,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 
   if (warp == 0) {
+    bool waited = false;
     if (lane == 0 && !*abort_flag) {
       const uint32_t tall_bytes = (uint32_t)((args.BH + 2) * args.BW * kBK * 2 + 3 * kBTileBytes);
       const uint32_t single_bytes = (uint32_t)(kATileBytes + kBTileBytes);
@@ -238,6 +246,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const KSeg sg = args.seg[si];
           const int nst = kseg_stages(sg);
           for (int js = max(0, kb_lo - g); js < nst && g + js < kb_hi; ++js) {
+            if (!waited) {
+              pdl_wait();
+              after_wait();
+              waited = true;
+            }
             if (q >= (uint32_t)STAGES && !mbar_wait(&empty_bar[s], ph ^ 1, abort_flag, args.err)) {
               ok = false;
               break;
@@ -270,6 +283,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+    }
+    if (lane == 0 && !waited) {
+      // no stage issued (no work unit, or the timeout test): wait all the same
+      pdl_wait();
+      after_wait();
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0 && !*abort_flag) {
@@ -346,6 +364,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const float* const colscale = args.epi.colscale;
     const double ln_inv = args.epi.ln_cols > 0 ? 1.0 / args.epi.ln_cols : 0.0;
     const float ln_eps = args.epi.ln_eps;
+    // 32-byte stores and residual loads when every row segment of a chunk starts on a
+    // 32-byte boundary (each thread writes a row: one sector per instruction)
+    const bool out32 = ((reinterpret_cast<uintptr_t>(out) | ((uintptr_t)ld_out * 2)) & 31) == 0;
+    const bool res32 = ((reinterpret_cast<uintptr_t>(residual) | ((uintptr_t)ld_res * 2)) & 31) == 0;
+    const bool f32out32 = partial ? (N % 8 == 0 && (reinterpret_cast<uintptr_t>(partial) & 31) == 0)
+                                  : (((reinterpret_cast<uintptr_t>(out) | ((uintptr_t)ld_out * 4)) & 31) == 0);
 
     const int et = threadIdx.x - 64;  // 0..255
     const int half = (warp - 2) >> 2;  // which alternate 32-column chunks this warp handles
@@ -443,7 +467,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (partial || f32_out) {
           float* dst = partial ? partial + ((size_t)z * Ho * Wo + grow) * N + nb
                                : reinterpret_cast<float*>(out) + grow * ld_out + nb;
-          if (full) {
+          if (full && f32out32) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              st_global_v8(dst + 8 * w, __float_as_uint(v[8 * w]), __float_as_uint(v[8 * w + 1]),
+                           __float_as_uint(v[8 * w + 2]), __float_as_uint(v[8 * w + 3]), __float_as_uint(v[8 * w + 4]),
+                           __float_as_uint(v[8 * w + 5]), __float_as_uint(v[8 * w + 6]), __float_as_uint(v[8 * w + 7]));
+          } else if (full) {
             float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
             for (int w = 0; w < 8; ++w) d4[w] = make_float4(v[4 * w], v[4 * w + 1], v[4 * w + 2], v[4 * w + 3]);
@@ -464,7 +494,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             o[j] = pack_bf16x2(a0, a1);
           }
           __nv_bfloat16* dst = out + grow * ld_out + (nb >> 1);
-          if (full) {
+          if (full && out32) {
+            st_global_v8(dst, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+          } else if (full) {
             uint4* d4 = reinterpret_cast<uint4*>(dst);
             d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
             d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
@@ -481,7 +513,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         if (residual) {
           const __nv_bfloat16* rs = residual + grow * ld_res + nb;
-          if (full) {
+          if (full && res32) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t w[8];
+              ld_global_v8(rs + 16 * h, w);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                v[16 * h + 2 * i] += bf16lo(w[i]);
+                v[16 * h + 2 * i + 1] += bf16hi(w[i]);
+              }
+            }
+          } else if (full) {
             const uint4* r4 = reinterpret_cast<const uint4*>(rs);
 #pragma unroll
             for (int w4 = 0; w4 < 4; ++w4) {
@@ -504,18 +547,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         __nv_bfloat16* dst = out + grow * ld_out + nb;
         if (full && f16_begin > 0 && nb >= f16_begin) {
           // FP16 columns (the attention values V; no row statistics are taken over them)
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
+          uint32_t o[16];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            d4[w] = make_uint4(pack_f16x2(v[8 * w + 0], v[8 * w + 1]), pack_f16x2(v[8 * w + 2], v[8 * w + 3]),
-                               pack_f16x2(v[8 * w + 4], v[8 * w + 5]), pack_f16x2(v[8 * w + 6], v[8 * w + 7]));
+          for (int i = 0; i < 16; ++i) o[i] = pack_f16x2(v[2 * i], v[2 * i + 1]);
+          if (out32) {
+            st_global_v8(dst, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+            st_global_v8(dst + 16, o[8], o[9], o[10], o[11], o[12], o[13], o[14], o[15]);
+          } else {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) d4[w] = make_uint4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
           }
         } else if (full) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
+          uint32_t o[16];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            d4[w] = make_uint4(pack_bf16x2(v[8 * w + 0], v[8 * w + 1]), pack_bf16x2(v[8 * w + 2], v[8 * w + 3]),
-                               pack_bf16x2(v[8 * w + 4], v[8 * w + 5]), pack_bf16x2(v[8 * w + 6], v[8 * w + 7]));
+          for (int i = 0; i < 16; ++i) o[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          if (out32) {
+            st_global_v8(dst, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+            st_global_v8(dst + 16, o[8], o[9], o[10], o[11], o[12], o[13], o[14], o[15]);
+          } else {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) d4[w] = make_uint4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
           }
           if (rowstat_out) {
 #pragma unroll
