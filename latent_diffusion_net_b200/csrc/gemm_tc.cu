@@ -436,11 +436,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tc_fence_before();
         asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
       }
+      // TMEM reads run one chunk ahead of the arithmetic and stores
+      uint32_t rn[32];
+      if (half < kChunks) tmem_ld_32x32b_x32(tacc + half * 32, rn);
 #pragma unroll 1
       for (int cc = half; cc < kChunks; cc += 2) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tacc + cc * 32, r);
-        tmem_ld_wait();
+        tmem_ld_wait_regs(rn);
+        float v[32];
+        {
+          const uint32_t ecol_s = smem_u32(ecol + cc * 32), escl_s = smem_u32(escl + cc * 32);
+          if (rowstat_in) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 sc = lds_f4(escl_s + 4 * j);
+              const float4 co = has_cols ? lds_f4(ecol_s + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+              v[j] = fmaf(ln_a, __uint_as_float(rn[j]), fmaf(ln_b, sc.x, co.x));
+              v[j + 1] = fmaf(ln_a, __uint_as_float(rn[j + 1]), fmaf(ln_b, sc.y, co.y));
+              v[j + 2] = fmaf(ln_a, __uint_as_float(rn[j + 2]), fmaf(ln_b, sc.z, co.z));
+              v[j + 3] = fmaf(ln_a, __uint_as_float(rn[j + 3]), fmaf(ln_b, sc.w, co.w));
+            }
+          } else if (has_cols) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 co = lds_f4(ecol_s + 4 * j);
+              v[j] = __uint_as_float(rn[j]) + co.x;
+              v[j + 1] = __uint_as_float(rn[j + 1]) + co.y;
+              v[j + 2] = __uint_as_float(rn[j + 2]) + co.z;
+              v[j + 3] = __uint_as_float(rn[j + 3]) + co.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rn[j]);
+          }
+        }
+        if (cc + 2 < kChunks) tmem_ld_32x32b_x32(tacc + (cc + 2) * 32, rn);
         if (cc + 2 >= kChunks) {
           // this warp's last read of the accumulator: once all epilogue warps
           // are here it goes back to the MMA issuer
@@ -451,18 +480,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (!valid) continue;
         const int nb = n0 + cc * 32;
         if (nb >= N) continue;
-        float v[32];
-        if (rowstat_in) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            v[j] = fmaf(ln_a, __uint_as_float(r[j]), fmaf(ln_b, escl[cc * 32 + j], has_cols ? ecol[cc * 32 + j] : 0.f));
-        } else if (has_cols) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + ecol[cc * 32 + j];
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        }
         const bool full = (nb + 32 <= N);
         if (partial || f32_out) {
           float* dst = partial ? partial + ((size_t)z * Ho * Wo + grow) * N + nb
@@ -571,11 +588,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             for (int w = 0; w < 4; ++w) d4[w] = make_uint4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
           }
           if (rowstat_out) {
+            // sums of the stored BF16 values, read back from the packed words
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float q = __bfloat162float(__float2bfloat16_rn(v[j]));
-              rs1 += q;
-              rs2 = fmaf(q, q, rs2);
+            for (int i = 0; i < 16; ++i) {
+              const float lo = bf16lo(o[i]), hi = bf16hi(o[i]);
+              rs1 += lo + hi;
+              rs2 = fmaf(lo, lo, fmaf(hi, hi, rs2));
             }
           }
         } else {
