@@ -149,6 +149,24 @@ def measured_traffic(kernel, workload_name):
         return None
 
 
+def ncu_family_shares(workload_name):
+    """Per-family shares of the step's device time from the committed ncu launch list
+    of this workload (uninstrumented: gpu__time_duration.sum of every launch), or {}."""
+    path = os.path.join(ROOT, "profiles", f"launches_{workload_name}.md")
+    keys = {"GEMM": "gemm_tc", "attention": "attention", "GroupNorm": "groupnorm", "other": "other"}
+    out = {}
+    try:
+        for line in open(path):
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            if len(cells) == 4 and cells[3].endswith("%"):
+                head = cells[0].split(" (")[0]
+                if head in keys:
+                    out[keys[head]] = float(cells[3][:-1]) / 100.0
+    except OSError:
+        return {}
+    return out
+
+
 def cpu_model():
     try:
         for line in open("/proc/cpuinfo"):
@@ -654,10 +672,19 @@ def main():
         roof = {"kernel": dom_name, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": None, "peak_source": f"{peak_src} HBM copy",
                 "launches_per_step": dom["launches"], "avg_launch_us": avg_ms * 1e3}
+    shares = ncu_family_shares(spec["name"])
+    if shares and dom_name in shares:
+        # the family's share of the uninstrumented launch list applied to the headline step time
+        ms_fam = shares[dom_name] * ms_step
+        if roof.get("bound") == "tensor":
+            roof["achieved_ncu_share"] = dom["flops"] / (ms_fam * 1e-3) / 1e12
+            roof["frac_ncu_share"] = roof["achieved_ncu_share"] / peak_tf
+        roof["ncu_share_source"] = f"profiles/launches_{spec['name']}.md"
     breakdown = {k: {"ms": round(v["ms"], 4), "share": round(v["ms"] / step_kernel_ms, 4), "launches": v["launches"],
                      "ms_in_step": round(v["ms"] / step_kernel_ms * ms_step, 4),
                      "tflops": round(v["flops"] / (v["ms"] * 1e-3) / 1e12, 1) if v["flops"] and v["ms"] > 0 else None,
-                     "gbs": round(v["bytes"] / (v["ms"] * 1e-3) / 1e9, 1) if v["ms"] > 0 else None}
+                     "gbs": round(v["bytes"] / (v["ms"] * 1e-3) / 1e9, 1) if v["ms"] > 0 else None,
+                     "ncu_share": shares.get(k)}
                  for k, v in sorted(fam.items(), key=lambda kv: -kv[1]["ms"])}
 
     # ------------------------------------------------------------- end to end through the ABI

@@ -82,6 +82,16 @@ def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch)
     assert bench.measured_traffic("missing", "sd21_base_unet_step_96") is None
 
 
+def test_ncu_family_shares_of_the_committed_launch_list():
+    """The uninstrumented per-family shares bench.py applies to the headline come
+    from the committed ncu launch list of the workload, and cover the whole step."""
+    shares = bench.ncu_family_shares("sd21_base_unet_step_96")
+    assert set(shares) == {"gemm_tc", "attention", "groupnorm", "other"}
+    assert abs(sum(shares.values()) - 1.0) < 0.01
+    assert shares["gemm_tc"] > shares["attention"] > shares["groupnorm"]
+    assert bench.ncu_family_shares("no_such_workload") == {}
+
+
 def test_peak_choice_follows_region_length_and_power_cap():
     peaks = {"bf16_tflops": 1674.6, "bf16_tflops_sustained": 1363.4, "hbm_gbs": 6547.5}
     assert bench.choose_peak(peaks, "measured", 0.12, {"reasons": []})[0] == 1674.6
