@@ -1,4 +1,4 @@
-"""The five synthetic workloads (shapes, seeds, value distributions).
+"""The synthetic workloads (shapes, seeds, value distributions).
 
 Every input is N(0, 1) rounded to BF16; every convolution/linear weight and
 bias is N(0, 1/fan_in) rounded to BF16; norm gains are 1 and shifts 0; the
