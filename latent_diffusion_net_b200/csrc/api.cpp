@@ -419,8 +419,17 @@ int run_attn(const Ctx& c, const bf16* qbase, int q_ld, int q_col, const bf16* k
 }
 
 // Transformer2DModel; y may alias x.
+// The context K/V of every cross-attention of a model, projected by one GEMM at
+// the start of the step: [ctx_len, ld] with the K columns of all blocks first and
+// their V columns (FP16) from v_begin on; block b reads K at b.ctx_k_col.
+struct CtxKV {
+  const bf16* kv;
+  int ld, v_begin;
+};
+
 sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int Wd, const bf16* x, const bf16* ctx,
-                          int ctx_len, int G, float gn_eps, float ln_eps, bf16* y, const TxScratch& s) {
+                          int ctx_len, int G, float gn_eps, float ln_eps, bf16* y, const TxScratch& s,
+                          const CtxKV* pre = nullptr) {
   const int HW = H * Wd;
   const int C = w.C;
   const int heads = C / 64;
@@ -506,10 +515,16 @@ sd_status run_transformer(const Ctx& c, const TxW& w, const void* pw, int H, int
           SD_OK)
         return r;
     }
-    if ((r = run_linear(c, ctx, ctx_len, w.ctx_dim, W(pw, b.kv2), 2 * C, nullptr, nullptr, 0, s.kv, 2 * C,
-                        sdk::GEMM_PLAIN, 0, nullptr, C)) != SD_OK)  // V as FP16
-      return r;
-    CK(run_attn(c, s.big, C, 0, s.kv, 2 * C, 0, C, s.ao, C, HW, ctx_len, heads));
+    if (b.kv2 >= 0) {
+      if ((r = run_linear(c, ctx, ctx_len, w.ctx_dim, W(pw, b.kv2), 2 * C, nullptr, nullptr, 0, s.kv, 2 * C,
+                          sdk::GEMM_PLAIN, 0, nullptr, C)) != SD_OK)  // V as FP16
+        return r;
+      CK(run_attn(c, s.big, C, 0, s.kv, 2 * C, 0, C, s.ao, C, HW, ctx_len, heads));
+    } else {
+      if (!pre || b.ctx_k_col < 0) return SD_ERR_UNSUPPORTED;
+      CK(run_attn(c, s.big, C, 0, pre->kv, pre->ld, b.ctx_k_col, pre->v_begin + b.ctx_k_col, s.ao, C, HW, ctx_len,
+                  heads));
+    }
     if ((r = record("attn2", s.ao, C, b.o2w, b.o2b)) != SD_OK) return r;
     {
       const LnFold f = producer();
@@ -842,6 +857,8 @@ struct UNetPlan {
   TxScratch ts;
   bf16* conv_scratch;
   bf16 *mid_a, *mid_b;
+  bf16* ctx_kv;     // [ctx_len, 2 * ctx_k_cols]: the context K/V of every cross-attention
+  int ctx_k_cols;
 };
 
 size_t plan_unet(Arena& ar, const sd_unet_cfg* cfg, cudaStream_t st, int sms, UNetPlan* p) {
@@ -856,6 +873,12 @@ size_t plan_unet(Arena& ar, const sd_unet_cfg* cfg, cudaStream_t st, int sms, UN
     p->add_x = ar.f32((size_t)cfg->add_text_dim + (size_t)cfg->add_time_ids * cfg->add_time_dim);
     p->add_h = ar.f32(cfg->temb_dim);
   }
+  // K width of the context K/V matrix: C per BasicTransformer block of every cross-attention
+  int kcols = cfg->mid_depth * ch[L - 1];
+  for (int l = 0; l < L; ++l)
+    if (cfg->attn_depth[l] > 0) kcols += (2 * cfg->layers_per_block + 1) * cfg->attn_depth[l] * ch[l];
+  p->ctx_k_cols = kcols;
+  p->ctx_kv = ar.bf((size_t)cfg->ctx_len * 2 * kcols);
   int64_t tsum = 0;
   for (int l = 0; l < L; ++l) tsum += (int64_t)ch[l] * (2 * cfg->layers_per_block + 1);
   tsum += 2 * ch[L - 1];
@@ -1339,6 +1362,12 @@ sd_status sd_unet_step_cond(const sd_unet_cfg* cfg, const void* pw, const void* 
   const bf16* ctx = static_cast<const bf16*>(context);
   uint8_t* shared = reinterpret_cast<uint8_t*>(p.conv_scratch);
 
+  // the context K/V of every cross-attention in one GEMM (the context is the same for all of them)
+  if (u.ctx_kv_w < 0 || u.ctx_k_cols != p.ctx_k_cols) return SD_ERR_UNSUPPORTED;
+  if ((s = run_linear(c, ctx, cfg->ctx_len, cfg->ctx_dim, W(pw, u.ctx_kv_w), 2 * p.ctx_k_cols, nullptr, nullptr, 0,
+                      p.ctx_kv, 2 * p.ctx_k_cols, sdk::GEMM_PLAIN, 0, nullptr, p.ctx_k_cols)) != SD_OK)  // V as FP16
+    return s;
+  const CtxKV pre{p.ctx_kv, 2 * p.ctx_k_cols, p.ctx_k_cols};
   // time embedding and every resblock's projection of SiLU(temb), batched
   if ((s = run_time(c, u.time, pw, cfg->time_proj_dim, cfg->temb_dim, timestep, p.phi, p.hid, p.temb)) != SD_OK)
     return s;
@@ -1411,7 +1440,7 @@ sd_status sd_unet_step_cond(const sd_unet_cfg* cfg, const void* pw, const void* 
         return s;
       if (!lv.attn.empty()) {
         TxScratch ts = carve_tx(shared, H * Wd, ch[l], cfg->ctx_len);
-        if ((s = run_transformer(c, lv.attn[i], pw, H, Wd, dst, ctx, cfg->ctx_len, G, eps, eps, dst, ts)) != SD_OK)
+        if ((s = run_transformer(c, lv.attn[i], pw, H, Wd, dst, ctx, cfg->ctx_len, G, eps, eps, dst, ts, &pre)) != SD_OK)
           return s;
       }
       h = dst;
@@ -1431,7 +1460,7 @@ sd_status sd_unet_step_cond(const sd_unet_cfg* cfg, const void* pw, const void* 
     if ((s = run_resblock(c, u.mid_res0, pw, H, Wd, h, hc, nullptr, 0, tproj[ri++], G, eps, p.mid_a, rs)) != SD_OK)
       return s;
     TxScratch ts = carve_tx(shared, H * Wd, hc, cfg->ctx_len);
-    if ((s = run_transformer(c, u.mid_attn, pw, H, Wd, p.mid_a, ctx, cfg->ctx_len, G, eps, eps, p.mid_a, ts)) !=
+    if ((s = run_transformer(c, u.mid_attn, pw, H, Wd, p.mid_a, ctx, cfg->ctx_len, G, eps, eps, p.mid_a, ts, &pre)) !=
         SD_OK)
       return s;
     if ((s = run_resblock(c, u.mid_res1, pw, H, Wd, p.mid_a, hc, nullptr, 0, tproj[ri++], G, eps, p.mid_b, rs)) !=
@@ -1454,7 +1483,7 @@ sd_status sd_unet_step_cond(const sd_unet_cfg* cfg, const void* pw, const void* 
       if ((s = run_resblock(c, lv.res[i], pw, H, Wd, h, hc, sk, cs, tproj[ri++], G, eps, dst, rs)) != SD_OK) return s;
       if (!lv.attn.empty()) {
         TxScratch ts = carve_tx(shared, H * Wd, ch[l], cfg->ctx_len);
-        if ((s = run_transformer(c, lv.attn[i], pw, H, Wd, dst, ctx, cfg->ctx_len, G, eps, eps, dst, ts)) != SD_OK)
+        if ((s = run_transformer(c, lv.attn[i], pw, H, Wd, dst, ctx, cfg->ctx_len, G, eps, eps, dst, ts, &pre)) != SD_OK)
           return s;
       }
       h = dst;

@@ -30,6 +30,32 @@ int64_t Table::add(const std::string& name, std::initializer_list<int64_t> shape
   return x.packed_off;
 }
 
+int Table::add_deferred(const std::string& name, std::initializer_list<int64_t> shape, int kind, int fan_in) {
+  Tensor x;
+  x.name = name;
+  x.ndim = (int)shape.size();
+  int i = 0;
+  for (int64_t s : shape) x.shape[i++] = s;
+  x.kind = kind;
+  x.fan_in = fan_in;
+  x.canon_off = canon_elems;
+  canon_elems += x.numel();
+  x.packed_elems = x.numel();
+  x.packed_off = -1;
+  t.push_back(x);
+  return (int)t.size() - 1;
+}
+
+int64_t Table::place_run(const std::vector<int>& idx) {
+  packed_bytes = (packed_bytes + 255) & ~int64_t(255);
+  const int64_t first = packed_bytes;
+  for (int i : idx) {
+    t[i].packed_off = packed_bytes;
+    packed_bytes += t[i].packed_elems * 2;
+  }
+  return first;
+}
+
 int64_t Table::add_derived(const Derived& x0) {
   Derived x = x0;
   packed_bytes = (packed_bytes + 255) & ~int64_t(255);
@@ -95,7 +121,7 @@ ResW add_resblock(Table& tab, const std::string& p, int ci, int co, int temb) {
   return w;
 }
 
-TxW add_transformer(Table& tab, const std::string& p, int C, int depth, int D) {
+TxW add_transformer(Table& tab, const std::string& p, int C, int depth, int D, CtxKVGather* gather) {
   TxW w;
   w.C = C;
   w.depth = depth;
@@ -124,9 +150,18 @@ TxW add_transformer(Table& tab, const std::string& p, int C, int depth, int D) {
     const int ln2b = tab.last();
     k.q2 = tab.add(b + ".attn2.q.weight", {C, C}, SD_KIND_WEIGHT, C, PACK_LNFOLD, ln2g);
     const int q2 = tab.last();
-    // k, v of the cross-attention are consecutive: one [2C, D] matrix
-    k.kv2 = tab.add(b + ".attn2.k.weight", {C, D}, SD_KIND_WEIGHT, D);
-    tab.add(b + ".attn2.v.weight", {C, D}, SD_KIND_WEIGHT, D);
+    if (gather) {
+      // placed with every other block's K (and V) by the caller
+      k.kv2 = -1;
+      k.ctx_k_col = gather->cols;
+      gather->cols += C;
+      gather->k.push_back(tab.add_deferred(b + ".attn2.k.weight", {C, D}, SD_KIND_WEIGHT, D));
+      gather->v.push_back(tab.add_deferred(b + ".attn2.v.weight", {C, D}, SD_KIND_WEIGHT, D));
+    } else {
+      // k, v of the cross-attention are consecutive: one [2C, D] matrix
+      k.kv2 = tab.add(b + ".attn2.k.weight", {C, D}, SD_KIND_WEIGHT, D);
+      tab.add(b + ".attn2.v.weight", {C, D}, SD_KIND_WEIGHT, D);
+    }
     k.o2w = tab.add(b + ".attn2.out.weight", {C, C}, SD_KIND_WEIGHT, C);
     k.o2b = tab.add(b + ".attn2.out.bias", {C}, SD_KIND_BIAS, C);
     k.ln3g = tab.add(b + ".ln3.gamma", {C}, SD_KIND_NORM_GAMMA, 0);
@@ -155,6 +190,7 @@ TxW add_transformer(Table& tab, const std::string& p, int C, int depth, int D) {
 
 UNetW add_unet(Table& tab, const sd_unet_cfg& cfg) {
   UNetW u;
+  CtxKVGather gather;
   const int L = cfg.n_levels;
   const int* ch = cfg.block_channels;
   u.time = add_time(tab, "time", cfg.time_proj_dim, cfg.temb_dim);
@@ -172,7 +208,8 @@ UNetW add_unet(Table& tab, const sd_unet_cfg& cfg) {
       lv.res.push_back(add_resblock(tab, p + ".res." + std::to_string(i), c_prev, ch[l], cfg.temb_dim));
       c_prev = ch[l];
       if (cfg.attn_depth[l] > 0)
-        lv.attn.push_back(add_transformer(tab, p + ".attn." + std::to_string(i), ch[l], cfg.attn_depth[l], cfg.ctx_dim));
+        lv.attn.push_back(
+            add_transformer(tab, p + ".attn." + std::to_string(i), ch[l], cfg.attn_depth[l], cfg.ctx_dim, &gather));
       skips.push_back(ch[l]);
     }
     lv.has_down = l < L - 1;
@@ -183,7 +220,7 @@ UNetW add_unet(Table& tab, const sd_unet_cfg& cfg) {
     u.down.push_back(lv);
   }
   u.mid_res0 = add_resblock(tab, "mid.res.0", ch[L - 1], ch[L - 1], cfg.temb_dim);
-  u.mid_attn = add_transformer(tab, "mid.attn.0", ch[L - 1], cfg.mid_depth, cfg.ctx_dim);
+  u.mid_attn = add_transformer(tab, "mid.attn.0", ch[L - 1], cfg.mid_depth, cfg.ctx_dim, &gather);
   u.mid_res1 = add_resblock(tab, "mid.res.1", ch[L - 1], ch[L - 1], cfg.temb_dim);
   c_prev = ch[L - 1];
   for (int up = 0; up < L; ++up) {
@@ -196,13 +233,20 @@ UNetW add_unet(Table& tab, const sd_unet_cfg& cfg) {
       lv.res.push_back(add_resblock(tab, p + ".res." + std::to_string(i), c_prev + cs, ch[l], cfg.temb_dim));
       c_prev = ch[l];
       if (cfg.attn_depth[l] > 0)
-        lv.attn.push_back(add_transformer(tab, p + ".attn." + std::to_string(i), ch[l], cfg.attn_depth[l], cfg.ctx_dim));
+        lv.attn.push_back(
+            add_transformer(tab, p + ".attn." + std::to_string(i), ch[l], cfg.attn_depth[l], cfg.ctx_dim, &gather));
     }
     lv.has_up = up < L - 1;
     if (lv.has_up) lv.up = add_conv3x3(tab, "up." + std::to_string(up) + ".up", ch[l], ch[l]);
     u.up.push_back(lv);
   }
   u.out = add_output(tab, ch[0], cfg.out_channels);
+  if (!gather.k.empty()) {
+    // [K of every cross-attention | V of every cross-attention], one row per output feature
+    u.ctx_kv_w = tab.place_run(gather.k);
+    tab.place_run(gather.v);
+    u.ctx_k_cols = gather.cols;
+  }
   return u;
 }
 

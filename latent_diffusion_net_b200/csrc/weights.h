@@ -62,6 +62,12 @@ struct Table {
               int pack = PACK_COPY, int aux = 0);
   // Appends a derived FP32 vector of `rows` entries; returns its packed byte offset.
   int64_t add_derived(const Derived& x);
+  // Appends a tensor whose packed place is given later by place_run (canonical
+  // order is unchanged); returns its index.
+  int add_deferred(const std::string& name, std::initializer_list<int64_t> shape, int kind, int fan_in);
+  // Places the deferred tensors `idx` back to back (one matrix when they share
+  // their row length and each is a multiple of 256 bytes); returns the offset of the first.
+  int64_t place_run(const std::vector<int>& idx);
   int last() const { return (int)t.size() - 1; }
 };
 
@@ -80,7 +86,10 @@ struct ResW {
   int64_t n1g, n1b, c1w, c1b, tw, tb, n2g, n2b, c2w, c2b, sw, sb;  // sw/sb = -1 without shortcut
 };
 struct TxBlockW {
+  // kv2 = -1 when the cross-attention K/V weights live in the whole model's context
+  // K/V matrix instead (ctx_k_col = this block's first K column there)
   int64_t ln1g, ln1b, qkv, o1w, o1b, ln2g, ln2b, q2, kv2, o2w, o2b, ln3g, ln3b, f1w, f1b, f2w, f2b;
+  int ctx_k_col = -1;
   // LayerNorm folded into the following linear: qkv, q2 and f1w are packed as
   // W * gamma; c1 / c2 are the FP32 column terms of the GEMM epilogue
   int64_t qkv_c1, qkv_c2, q2_c1, q2_c2, f1_c1, f1_c2;
@@ -96,10 +105,21 @@ ConvW add_conv3x3(Table& tab, const std::string& prefix, int c_in, int c_out);
 ConvW add_conv_in(Table& tab, const std::string& prefix, int c_in, int c_out, int kp);
 OutW add_output(Table& tab, int c_in, int c_out);
 ResW add_resblock(Table& tab, const std::string& prefix, int c_in, int c_out, int temb_dim);
-TxW add_transformer(Table& tab, const std::string& prefix, int C, int depth, int ctx_dim);
+// The context K/V weights of every cross-attention of a model, gathered into one
+// [K of all blocks | V of all blocks] x ctx_dim matrix so that one GEMM projects
+// the context for all of them: `k`/`v` collect the deferred tensors, `cols` the K width.
+struct CtxKVGather {
+  std::vector<int> k, v;
+  int cols = 0;
+};
+TxW add_transformer(Table& tab, const std::string& prefix, int C, int depth, int ctx_dim,
+                    CtxKVGather* gather = nullptr);
 
 // Whole U-Net: module order follows the forward pass.
 struct UNetW {
+  // context K/V of all cross-attentions: [2 * ctx_k_cols, ctx_dim] at ctx_kv_w (K rows first)
+  int64_t ctx_kv_w = -1;
+  int ctx_k_cols = 0;
   TimeW time;
   bool has_add;  // SDXL added conditioning MLP (same shape as the time MLP)
   TimeW add;
