@@ -630,15 +630,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 // rs1 / rs2, the sums of the stored BF16 values (plain stores only).
 __device__ __forceinline__ void splitk_reduce_vec(const float* __restrict__ partial, int splits, int M, int N,
                                                   const GemmEpi& epi, int row, int c, float& rs1, float& rs2) {
-  float v[8];
-  const float4* p0 = reinterpret_cast<const float4*>(partial + (size_t)row * N + c);
-  float4 a = p0[0], b = p0[1];
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  for (int z = 1; z < splits; ++z) {
-    const float4* pz = reinterpret_cast<const float4*>(partial + ((size_t)z * M + row) * N + c);
-    a = pz[0];
-    b = pz[1];
-    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w; v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  // the splits' partials are requested four at a time before any is added; the
+  // sum still runs in split order, so the result does not depend on the grouping
+  float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const size_t zstride = (size_t)M * N;
+  const float* base = partial + (size_t)row * N + c;
+  for (int z0 = 0; z0 < splits; z0 += 4) {
+    float4 a[4], b[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (z0 + u < splits) {
+        const float4* pz = reinterpret_cast<const float4*>(base + (size_t)(z0 + u) * zstride);
+        a[u] = __ldcg(pz);
+        b[u] = __ldcg(pz + 1);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (z0 + u < splits) {
+        if (z0 + u == 0) {
+          v[0] = a[u].x; v[1] = a[u].y; v[2] = a[u].z; v[3] = a[u].w;
+          v[4] = b[u].x; v[5] = b[u].y; v[6] = b[u].z; v[7] = b[u].w;
+        } else {
+          v[0] += a[u].x; v[1] += a[u].y; v[2] += a[u].z; v[3] += a[u].w;
+          v[4] += b[u].x; v[5] += b[u].y; v[6] += b[u].z; v[7] += b[u].w;
+        }
+      }
+    }
   }
   if (epi.rowstat_in) {
     // folded LayerNorm: rstd * acc - rstd * mean * colscale + colvec
