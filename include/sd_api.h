@@ -220,6 +220,11 @@ enum { SD_CONV_IN = 0, SD_CONV_DOWNSAMPLE = 1, SD_CONV_UPSAMPLE = 2, SD_CONV_OUT
  *   - after each block's tensors come two derived FP32 vectors per such layer:
  *     c1 = row sums of W' and c2 = W * beta + bias, which the GEMM epilogue uses
  *     to apply the LayerNorm from per-row statistics (no LayerNorm kernel runs);
+ *   - in a whole U-Net (sd_unet_pack_weights) the cross-attention K and V weights
+ *     of every BasicTransformer block are placed last, out of table order, as one
+ *     [K of all blocks | V of all blocks] x ctx_dim matrix, so that one GEMM
+ *     projects the context for every cross-attention of the step (the
+ *     packed_offset of each tensor in sd_unet_weight_layout gives its place);
  *   - every other tensor is copied unchanged. */
 sd_status sd_time_pack_weights(const sd_time_cfg* cfg, const uint16_t* canonical, void* packed);
 sd_status sd_conv_pack_weights(const sd_conv_cfg* cfg, int32_t conv_kind, const uint16_t* canonical,
