@@ -104,6 +104,26 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction (sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+
+// (x0, x1) = (s0 * k + c, s1 * k + c) as one packed FP32 FMA (sm_100), each element
+// rounded exactly as a scalar fmaf
+__device__ __forceinline__ void fma2(float s0, float s1, float k, float c, float& x0, float& x1) {
+  asm("{\n\t.reg .b64 t, u, v;\n\t"
+      "mov.b64 t, {%2, %3};\n\t"
+      "mov.b64 u, {%4, %4};\n\t"
+      "mov.b64 v, {%5, %5};\n\t"
+      "fma.rn.f32x2 t, t, u, v;\n\t"
+      "mov.b64 {%0, %1}, t;\n\t}"
+      : "=f"(x0), "=f"(x1)
+      : "f"(s0), "f"(s1), "f"(k), "f"(c));
+}
+
 __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -363,13 +383,13 @@ __global__ void __launch_bounds__(192, 2)
         }
         float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 128; i += 4) {
-          m0 = fmaxf(m0, __uint_as_float(sv[i]));
-          m1 = fmaxf(m1, __uint_as_float(sv[i + 1]));
-          m2 = fmaxf(m2, __uint_as_float(sv[i + 2]));
-          m3 = fmaxf(m3, __uint_as_float(sv[i + 3]));
+        for (int i = 0; i < 128; i += 8) {
+          m0 = max3(m0, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+          m1 = max3(m1, __uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3]));
+          m2 = max3(m2, __uint_as_float(sv[i + 4]), __uint_as_float(sv[i + 5]));
+          m3 = max3(m3, __uint_as_float(sv[i + 6]), __uint_as_float(sv[i + 7]));
         }
-        mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        mx = max3(m0, m1, fmaxf(m2, m3));
       }
       // new running maximum; O is rescaled (after the wait below) only when it grew by more than 2^8
       float alpha = 1.f;
@@ -396,8 +416,8 @@ __global__ void __launch_bounds__(192, 2)
       for (int i = 0; i < 64; i += 4) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const float x0 = fmaf(__uint_as_float(sv[2 * (i + u)]), sl2, -m_used);
-          const float x1 = fmaf(__uint_as_float(sv[2 * (i + u) + 1]), sl2, -m_used);
+          float x0, x1;
+          fma2(__uint_as_float(sv[2 * (i + u)]), __uint_as_float(sv[2 * (i + u) + 1]), sl2, -m_used, x0, x1);
           pk[i + u] = ex2_f16x2(cvt_f16x2(x0, x1));
         }
         hs0 = add_f16x2(hs0, pk[i]);
