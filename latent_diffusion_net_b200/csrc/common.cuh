@@ -63,6 +63,30 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
 
+// Packed FP32 pairs (sm_100): each element rounded exactly as the scalar operation.
+// (y0, y1) = (a0 + b0, a1 + b1)
+__device__ __forceinline__ void add2(float a0, float a1, float b0, float b1, float& y0, float& y1) {
+  asm("{\n\t.reg .b64 p, q;\n\t"
+      "mov.b64 p, {%2, %3};\n\t"
+      "mov.b64 q, {%4, %5};\n\t"
+      "add.rn.f32x2 p, p, q;\n\t"
+      "mov.b64 {%0, %1}, p;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// (y0, y1) = (a0 * b0 + c0, a1 * b1 + c1)
+__device__ __forceinline__ void fma2v(float a0, float a1, float b0, float b1, float c0, float c1, float& y0,
+                                      float& y1) {
+  asm("{\n\t.reg .b64 p, q, r;\n\t"
+      "mov.b64 p, {%2, %3};\n\t"
+      "mov.b64 q, {%4, %5};\n\t"
+      "mov.b64 r, {%6, %7};\n\t"
+      "fma.rn.f32x2 p, p, q, r;\n\t"
+      "mov.b64 {%0, %1}, p;\n\t}"
+      : "=f"(y0), "=f"(y1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
 __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));

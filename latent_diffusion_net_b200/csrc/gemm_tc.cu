@@ -450,19 +450,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             for (int j = 0; j < 32; j += 4) {
               const float4 sc = lds_f4(escl_s + 4 * j);
               const float4 co = has_cols ? lds_f4(ecol_s + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
-              v[j] = fmaf(ln_a, __uint_as_float(rn[j]), fmaf(ln_b, sc.x, co.x));
-              v[j + 1] = fmaf(ln_a, __uint_as_float(rn[j + 1]), fmaf(ln_b, sc.y, co.y));
-              v[j + 2] = fmaf(ln_a, __uint_as_float(rn[j + 2]), fmaf(ln_b, sc.z, co.z));
-              v[j + 3] = fmaf(ln_a, __uint_as_float(rn[j + 3]), fmaf(ln_b, sc.w, co.w));
+              float t0, t1, t2, t3;  // ln_b * colscale + colvec, then ln_a * acc + that
+              fma2v(ln_b, ln_b, sc.x, sc.y, co.x, co.y, t0, t1);
+              fma2v(ln_b, ln_b, sc.z, sc.w, co.z, co.w, t2, t3);
+              fma2v(ln_a, ln_a, __uint_as_float(rn[j]), __uint_as_float(rn[j + 1]), t0, t1, v[j], v[j + 1]);
+              fma2v(ln_a, ln_a, __uint_as_float(rn[j + 2]), __uint_as_float(rn[j + 3]), t2, t3, v[j + 2], v[j + 3]);
             }
           } else if (has_cols) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
               const float4 co = lds_f4(ecol_s + 4 * j);
-              v[j] = __uint_as_float(rn[j]) + co.x;
-              v[j + 1] = __uint_as_float(rn[j + 1]) + co.y;
-              v[j + 2] = __uint_as_float(rn[j + 2]) + co.z;
-              v[j + 3] = __uint_as_float(rn[j + 3]) + co.w;
+              add2(__uint_as_float(rn[j]), __uint_as_float(rn[j + 1]), co.x, co.y, v[j], v[j + 1]);
+              add2(__uint_as_float(rn[j + 2]), __uint_as_float(rn[j + 3]), co.z, co.w, v[j + 2], v[j + 3]);
             }
           } else {
 #pragma unroll
@@ -536,10 +535,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               uint32_t w[8];
               ld_global_v8(rs + 16 * h, w);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                v[16 * h + 2 * i] += bf16lo(w[i]);
-                v[16 * h + 2 * i + 1] += bf16hi(w[i]);
-              }
+              for (int i = 0; i < 8; ++i)
+                add2(v[16 * h + 2 * i], v[16 * h + 2 * i + 1], bf16lo(w[i]), bf16hi(w[i]), v[16 * h + 2 * i],
+                     v[16 * h + 2 * i + 1]);
             }
           } else if (full) {
             const uint4* r4 = reinterpret_cast<const uint4*>(rs);

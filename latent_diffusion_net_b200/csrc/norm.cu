@@ -42,6 +42,23 @@ __device__ __forceinline__ float silu_tanh(float x) {
   return fmaf(h, th, h);
 }
 
+// Normalise 8 channels (o = f * a + b, optional SiLU) in packed FP32 pairs; the
+// same arithmetic, element for element, as the scalar form.
+__device__ __forceinline__ void gn_norm8(float (&f)[8], const float (&a)[8], const float (&b)[8], int silu) {
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) fma2v(f[j], f[j + 1], a[j], a[j + 1], b[j], b[j + 1], f[j], f[j + 1]);
+  if (silu) {
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      float h0, h1, t0, t1;
+      fma2v(f[j], f[j + 1], 0.5f, 0.5f, 0.f, 0.f, h0, h1);  // 0.5 * x, exact
+      asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(h0));
+      asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(h1));
+      fma2v(h0, h1, t0, t1, h0, h1, f[j], f[j + 1]);
+    }
+  }
+}
+
 __global__ void gn_stats_kernel(const __nv_bfloat16* __restrict__ x0, int C0, const __nv_bfloat16* __restrict__ x1,
                                 int C1, int HW, int G, int ppi, unsigned long long* __restrict__ acc) {
   extern __shared__ float4 red[];  // [blockDim.x]
@@ -348,12 +365,7 @@ __global__ void __launch_bounds__(kGnThreads, 1)
     const uint4 wk = slice[k * blockDim.x + t];
     float f[8] = {bf16lo(wk.x), bf16hi(wk.x), bf16lo(wk.y), bf16hi(wk.y),
                   bf16lo(wk.z), bf16hi(wk.z), bf16lo(wk.w), bf16hi(wk.w)};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float o = fmaf(f[j], sc[j], sh[j]);
-      if (silu) o = silu_tanh(o);
-      f[j] = o;
-    }
+    gn_norm8(f, sc, sh, silu);
     *reinterpret_cast<uint4*>(yq + (size_t)k * ppi * C) =
         make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
   }
