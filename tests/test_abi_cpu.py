@@ -251,3 +251,42 @@ def test_vae_table_matches_oracle_and_validates():
     assert B.sd_vae_decode(B.vae_cfg(10, 10), fake, fake, fake, fake, 10 ** 10, check=False) == 3  # 100 tokens
     assert B.sd_vae_decode(B.vae_cfg(16, 16, groups=64), fake, fake, fake, fake, 10 ** 10, check=False) == 3
     assert B.sd_vae_decode(B.vae_cfg(16, 16), fake, None, fake, fake, 10 ** 10, check=False) == 1
+
+
+def test_sampler_schedules_and_validation_on_host():
+    """The host-side schedules of the sampling entry points equal the oracle's
+    (linear and cosine alpha_bar, float64), and the update and the loop reject
+    bad arguments before any launch."""
+    from oracle import sampler
+    lin = np.array(B.sd_schedule(B.SD_SCHED_LINEAR, 1000, 1e-4, 0.02))
+    np.testing.assert_allclose(lin, sampler.alphas_cumprod(sampler.linear_betas(1000, 1e-4, 0.02)), rtol=1e-12)
+    cos = np.array(B.sd_schedule(B.SD_SCHED_COSINE, 1000, 1e-4, 0.02))
+    np.testing.assert_allclose(cos, sampler.alphas_cumprod(sampler.cosine_betas(1000)), rtol=1e-12)
+    for args in [(B.SD_SCHED_LINEAR, 0, 1e-4, 0.02), (B.SD_SCHED_LINEAR, 1000, 0.02, 1e-4), (7, 1000, 1e-4, 0.02)]:
+        with pytest.raises(RuntimeError):
+            B.sd_schedule(*args)
+    fake = 1 << 20
+    ac = lin
+    ok = B.sampler_cfg(B.SD_SAMPLER_DDIM, 96 * 96 * 4, ac[499], ac[479], guidance=7.5)
+    assert B.sd_sampler_step(ok, None, fake, check=False) == 1                        # no state
+    assert B.sd_sampler_step(B.sampler_cfg(B.SD_SAMPLER_DDIM, 10, ac[499], ac[479]), fake, fake,
+                             check=False) == 2                                           # n % out_ch
+    assert B.sd_sampler_step(B.sampler_cfg(B.SD_SAMPLER_DDIM, 96 * 96 * 4, ac[499], ac[479], ld=2), fake, fake,
+                             x_bf16=fake, check=False) == 2                              # ld < out_ch
+    assert B.sd_sampler_step(ok, fake + 4, fake, check=False) == 4                    # misaligned
+    assert B.sd_sampler_step(B.sampler_cfg(B.SD_SAMPLER_DDIM, 96 * 96 * 4, ac[479], ac[499]), fake, fake,
+                             check=False) == 2                                           # alpha_bar_prev < alpha_bar_t
+    cfg = B.unet_cfg_from(model.SD21_BASE, 96, 96)
+    need = B.sd_denoise_workspace_size(cfg)
+    assert need > 2 * B.sd_unet_workspace_size(cfg)
+
+    def den(ts, kind=B.SD_SAMPLER_DDIM, ws_bytes=need, acs=ac, ctx=fake):
+        return B.sd_denoise(cfg, fake, kind, acs, ts, 7.5, fake, None, ctx, fake, None, None, None, None, fake,
+                            ws_bytes, check=False)
+
+    assert den([500, 500]) == 2          # timesteps must fall
+    assert den([1001]) == 2              # past T
+    assert den([]) == 2                  # no step
+    assert den([500], kind=5) == 3       # unknown sampler
+    assert den([500], ws_bytes=need - 1) == 5
+    assert den([500], ctx=None) == 1
