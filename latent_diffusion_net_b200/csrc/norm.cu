@@ -32,18 +32,11 @@ __device__ __forceinline__ long long to_fixed(float v, double scale) {
   return __double2ll_rn(d);
 }
 
-// SiLU(x) = x * sigmoid(x) = h + h * tanh(h) with h = x / 2: one MUFU operation
-// (tanh.approx, relative error about 2^-11) instead of an exponential and a
-// reciprocal; the normalise + SiLU pass is bound by that unit.
-__device__ __forceinline__ float silu_tanh(float x) {
-  const float h = 0.5f * x;
-  float th;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(h));
-  return fmaf(h, th, h);
-}
-
-// Normalise 8 channels (o = f * a + b, optional SiLU) in packed FP32 pairs; the
-// same arithmetic, element for element, as the scalar form.
+// Normalise 8 channels, o = f * a + b, in packed FP32 pairs (each element rounded
+// as the scalar fmaf), then optionally SiLU(o) = o * sigmoid(o) = h + h * tanh(h)
+// with h = o / 2: one MUFU operation (tanh.approx, relative error about 2^-11)
+// instead of an exponential and a reciprocal, since the normalise + SiLU pass is
+// bound by that unit.
 __device__ __forceinline__ void gn_norm8(float (&f)[8], const float (&a)[8], const float (&b)[8], int silu) {
 #pragma unroll
   for (int j = 0; j < 8; j += 2) fma2v(f[j], f[j + 1], a[j], a[j + 1], b[j], b[j + 1], f[j], f[j + 1]);
@@ -51,7 +44,7 @@ __device__ __forceinline__ void gn_norm8(float (&f)[8], const float (&a)[8], con
 #pragma unroll
     for (int j = 0; j < 8; j += 2) {
       float h0, h1, t0, t1;
-      fma2v(f[j], f[j + 1], 0.5f, 0.5f, 0.f, 0.f, h0, h1);  // 0.5 * x, exact
+      fma2v(f[j], f[j + 1], 0.5f, 0.5f, 0.f, 0.f, h0, h1);  // o / 2
       asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(h0));
       asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(h1));
       fma2v(h0, h1, t0, t1, h0, h1, f[j], f[j + 1]);
@@ -175,13 +168,14 @@ __global__ void gn_apply_kernel(const __nv_bfloat16* __restrict__ x0, int C0, co
     const int c = (int)(i % V) * 8;
     float f[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
                   bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+    float sc[8], sh[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float2 s = ab[c + j];
-      float o = fmaf(f[j], s.x, s.y);
-      if (silu) o = silu_tanh(o);
-      f[j] = o;
+      sc[j] = s.x;
+      sh[j] = s.y;
     }
+    gn_norm8(f, sc, sh, silu);
     *reinterpret_cast<uint4*>(y + (size_t)p * C + c) =
         make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
   };
