@@ -142,6 +142,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Bounded wait for a softmax warp. tcgen05.ld / tcgen05.st are warp-collective
+// (.sync.aligned): every lane of the warp must execute them together. The lanes
+// of one warp may leave the polling loop at different polls, and one lane may
+// give up while another sees the phase complete; the vote brings them back
+// together and gives all of them one answer, so the warp stays or leaves as a
+// whole.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort, int* err) {
+  const bool ok = mbar_wait(bar, parity, abort, err);
+  return __all_sync(0xffffffffu, ok);
+}
+
 struct __align__(64) AttnMaps {
   CUtensorMap q;
   CUtensorMap kv;
@@ -360,7 +371,7 @@ __global__ void __launch_bounds__(192, 2)
     for (int t = 0; t < T; ++t, j = (j + 1 == nt) ? 0 : j + 1) {
       const bool first = t == 0 || j == 0;
       const bool last = t == T - 1 || j == nt - 1;
-      if (!mbar_wait(s_full, t & 1, abort_flag, args.err)) break;
+      if (!mbar_wait_warp(s_full, t & 1, abort_flag, args.err)) break;
       tc_fence_after();
       const int kvalid = args.Nk - j * kAK;  // keys of this tile that exist
       // the whole S row into registers, then hand the TMEM columns back for S_{t+1}
@@ -426,9 +437,12 @@ __global__ void __launch_bounds__(192, 2)
         hs3 = add_f16x2(hs3, pk[i + 3]);
       }
       // the previous PV product must be done before P is overwritten or O rescaled
-      if (t > 0 && !mbar_wait(pv_done, (t - 1) & 1, abort_flag, args.err)) break;
+      if (t > 0 && !mbar_wait_warp(pv_done, (t - 1) & 1, abort_flag, args.err)) break;
       tc_fence_after();
-      if (rescale) {
+      // rows decide on their own whether O must be rescaled, but the TMEM round trip is
+      // warp-collective: the warp makes it when any of its rows needs it, and the rows
+      // that do not keep alpha = 1 (their O multiplied by 1, unchanged)
+      if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           uint32_t r[32];
@@ -460,7 +474,7 @@ __global__ void __launch_bounds__(192, 2)
       if (!last) continue;
 
       // ---------------------------------------------------------- end of this CTA's part of item X
-      if (!mbar_wait(pv_done, t & 1, abort_flag, args.err)) break;
+      if (!mbar_wait_warp(pv_done, t & 1, abort_flag, args.err)) break;
       tc_fence_after();
       {
         const int w_first = (int)cta_first_step(blockIdx.x, args.steps, args.ctas);  // recomputed: rarely needed

@@ -7,6 +7,8 @@ to the device once.
 """
 from __future__ import annotations
 
+from contextlib import nullcontext as _nullcontext
+
 import numpy as np
 import torch
 
@@ -142,8 +144,10 @@ class Workload:
         self.inputs = make_inputs(wid)
         self.dev_inputs = {k: to_dev_bf16(v, device) for k, v in self.inputs.items()}
         if s["kind"] == "denoise":
-            # the sampler's FP32 latent state, updated in place by every step
-            self.dev_inputs["x"] = torch.from_numpy(self.inputs["x"].reshape(-1).astype(np.float32)).to(device)
+            # the sampler's FP32 latent state, updated in place by every step, and the
+            # workload's latent it is reset to before each pass
+            self.x_init = torch.from_numpy(self.inputs["x"].reshape(-1).astype(np.float32)).to(device)
+            self.dev_inputs["x"] = self.x_init.clone()
             m = self.modules[0]
             m.ws_bytes = B.sd_denoise_workspace_size(self.cfg)
             m.ws = workspace(m.ws_bytes, device)
@@ -184,6 +188,13 @@ class Workload:
             return self.out
         if s["kind"] == "denoise":
             m = self.modules[0]
+            if latent is None:
+                # Every pass is the same guided step from the workload's latent. Chained
+                # passes would apply the step to its own output: with alpha_bar_prev = 1
+                # the state grows by 1/sqrt(alpha_bar_t) (3.6 at t = 500) per pass and
+                # within a few passes leaves the range of the fixed-point GroupNorm sums.
+                with torch.cuda.stream(stream) if isinstance(stream, torch.cuda.Stream) else _nullcontext():
+                    x.copy_(self.x_init)
             B.sd_denoise(self.cfg, m.packed_dev, B.SD_SAMPLER_DDIM, self.alphas_cumprod, [s["timestep"]],
                          s["guidance"], x, None, ctx, self.dev_inputs["ctx_uncond"], None, None, None, None, m.ws,
                          m.ws_bytes, stream)
