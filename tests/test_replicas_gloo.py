@@ -38,7 +38,8 @@ def _rank_main(rank, world, port, out):
 
 def test_two_ranks_take_the_slowest_time():
     world = 2
-    with mp.Manager() as mgr:
+    # the manager process is spawned too: forking a process whose BLAS threads are running can deadlock
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
