@@ -25,7 +25,9 @@
 //              kept in four packed FP16 partial sums per tile, added into FP32
 //              once per tile. The output O lives in TMEM and is rescaled only
 //              when the running maximum grew by more than 2^8 since the last
-//              rescale (P values stay <= 256).
+//              rescale (P values stay <= 256). The TMEM accesses are
+//              warp-collective, so a warp rescales together when any of its
+//              rows needs it (the others with factor 1).
 //   warp 4     TMA producer: Q once per item, K tiles (double-buffered) and V
 //              tiles (single buffer, reloaded once the previous PV product is
 //              done), zero-filled past the last key. V arrives as FP16 (the
