@@ -55,7 +55,7 @@ typedef enum {
   SD_OK = 0,
   SD_ERR_NULL_ARG = 1,             /* a required pointer is NULL */
   SD_ERR_BAD_SHAPE = 2,            /* inconsistent sizes, channel or context mismatch */
-  SD_ERR_UNSUPPORTED = 3,          /* batch != 1, head_dim != 64, C % 64 != 0, groups ... */
+  SD_ERR_UNSUPPORTED = 3,          /* batch != 1, head_dim != 64, C % 64 != 0, groups ..., device index >= 64 */
   SD_ERR_MISALIGNED = 4,           /* a device pointer is not 16-byte aligned */
   SD_ERR_WORKSPACE_TOO_SMALL = 5,  /* ws_bytes below sd_*_workspace_size() */
   SD_ERR_NOT_SM100 = 6,            /* current device is not compute capability 10.0 */

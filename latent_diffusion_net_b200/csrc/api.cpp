@@ -37,7 +37,8 @@ DevInfo g_dev[64];
 
 sd_status device_info(DevInfo* out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SD_ERR_LAUNCH;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return SD_ERR_LAUNCH;
+  if (dev >= 64) return SD_ERR_UNSUPPORTED;  // the per-device cache holds 64 devices
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DevInfo& d = g_dev[dev];
   if (!d.init) {
