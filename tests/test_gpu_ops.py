@@ -8,7 +8,6 @@ the bound per operator is 1e-2 and per block 2e-2."""
 import numpy as np
 import pytest
 
-import rescale_case
 from gpu_util import assert_close, chw, dev_np, hwc, oracle_params
 from oracle import model
 import oracle
@@ -167,30 +166,6 @@ def test_transformer(H, W, C, depth, D, L, affine):
     got = dev_np(y, (H, W, C))
     assert_close(got, ref, BLOCK_TOL)
     # the residual path dominates the output: also check the block's own contribution
-    assert_close(got - x, ref - chw(x).transpose(1, 2, 0), 3 * BLOCK_TOL)
-
-
-@pytest.mark.skip(reason="first run on a B200 pending: the warp-uniform O rescale this case drives is "
-                          "compiled but has not run on a GPU yet")
-@pytest.mark.parametrize("H,W,C,ctas", rescale_case.CASES)
-def test_transformer_rows_rescale_at_different_key_tiles(H, W, C, ctas):
-    """Self-attention Q/K weights doubled: query rows rescale their running output at
-    different key tiles, so the rows of one warp disagree (the CPU test of the case
-    counts those events). Whole items at 48x48x320, the split schedule and merge
-    kernel at 64x64x640."""
-    rows, canon = rescale_case.canonical(C)
-    cfg = B.transformer_cfg(H, W, C, 1, 77, 1024)
-    m = Hn.Module("attn", cfg)
-    m.load(canon)
-    p = oracle_params(rows, canon)
-    x, ctx = rescale_case.inputs(H, W, C)
-    y = torch.empty(H * W * C, dtype=torch.bfloat16, device="cuda")
-    B.sd_transformer_fwd(cfg, m.packed_dev, Hn.to_dev_bf16(x), Hn.to_dev_bf16(ctx), y, m.ws, m.ws_bytes)
-    torch.cuda.synchronize()
-    assert B.sd_query_device_status(m.ws) == 0
-    ref = hwc(oracle.transformer(chw(x), ctx, p, "t", 1))
-    got = dev_np(y, (H, W, C))
-    assert_close(got, ref, BLOCK_TOL)
     assert_close(got - x, ref - chw(x).transpose(1, 2, 0), 3 * BLOCK_TOL)
 
 
