@@ -38,8 +38,9 @@ DEFAULT_WORKLOAD = 5
 # the full-size guided DDIM step (two 96x96 denoiser passes and the update) stalled on
 # the GPU in eager and in graph runs. Its passes used to chain the step on its own output
 # until the activations overflowed, and the attention's O rescale then ran warp-collective
-# TMEM accesses in a diverged warp. Both are fixed, but the fix has not run on a GPU yet,
-# so the step stays out of the bench until a run confirms it
+# TMEM accesses in a diverged warp. Both are fixed (the rescale case of the GPU tests drives
+# the attention branch), but the full-size step has not been run again since, so it stays
+# out of the bench
 DISABLED = {9}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
